@@ -1,0 +1,483 @@
+#!/usr/bin/env python3
+"""Benchmark of the compressed-KV sparse decode-attention step on B200.
+
+One step = one pass of the whole decode path over a batch: for every layer, append the decode
+token through the compressor (position L-1; idempotent across steps), score every compressed
+entry and select the top-k (sparse layers), attend over the selected entries plus the window.
+Inputs are resident in HBM; L2 is flushed (256 MiB write) before every timed step, outside the
+step's events. The metric is decode-attention queries*layers per second over all ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ckv|reference]
+
+For N > 1 launch one rank per GPU with torch.distributed.run; every rank runs its own batch of
+the workload (data-parallel requests, no collective on the data path) and rank 0 prints one JSON
+line. `--impl reference` times the CPU oracle on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from synth import workloads as S  # noqa: E402
+
+METRIC = "decode attention queries*layers/s"
+UNIT = "queries*layers/s"
+DEFAULT_WORKLOAD = "csa_b8_ctx32k"
+FLUSH_BYTES = 256 << 20
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic bytes (per step, per layer), from the stored formats
+# ------------------------------------------------------------------------------------------------
+
+def entry_bytes(ls: S.LayerSpec, d: int) -> int:
+    return S.comp_code_bytes(ls.comp_dtype, d) + (d // 16 if ls.comp_dtype == "nvfp4" else 0)
+
+
+def token_bytes(ls: S.LayerSpec, d: int) -> int:
+    return S.win_code_bytes(ls.win_dtype, d) + (4 if ls.win_dtype == "fp8" else 0)
+
+
+def layer_bytes(w: S.Workload, ls: S.LayerSpec) -> dict:
+    """Bytes a step must move for one layer: the indexer reads every candidate once; attention
+    reads the selected entries, the window tokens, the query and writes the output; the append
+    reads the unfinished group's ring and writes one entry and one window token."""
+    d, h = w.head_dim, w.num_heads
+    idx_b = att_b = app_b = 0
+    for L in w.seq_lens:
+        n_c = L // ls.ratio
+        if ls.top_k is not None:
+            idx_b += n_c * entry_bytes(ls, d) + 4 * math.ceil(L / 256) + 4 * h * d
+            sel = min(ls.top_k, n_c)
+        else:
+            sel = n_c
+        att_b += sel * entry_bytes(ls, d) + min(w.window, L) * token_bytes(ls, d) + 2 * 4 * h * d
+        app_b += 4 * d + 4 + (ls.ratio - 1) * (4 * d + 4) + entry_bytes(ls, d) + token_bytes(ls, d)
+    return {"indexer": idx_b, "attention": att_b, "append": app_b}
+
+
+# ------------------------------------------------------------------------------------------------
+# environment
+# ------------------------------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap,power.draw")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:6]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def traffic_record(kernel: str, workload: str):
+    """dram bytes per launch of `kernel` from the committed ncu summary, if the kernel source
+    has not changed since it was captured (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"source_sha256:\s*([0-9a-f]+)", txt)
+    src = re.search(r"source_file:\s*(\S+)", txt)
+    if not (m and h and src):
+        return None
+    try:
+        cur = hashlib.sha256(open(os.path.join(ROOT, src.group(1)), "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return float(m.group(1)) if cur == h.group(1) else None
+
+
+# ------------------------------------------------------------------------------------------------
+# CUDA arm
+# ------------------------------------------------------------------------------------------------
+
+class Step:
+    """All layers of a workload on one GPU, with the step's inputs resident in HBM."""
+
+    def __init__(self, ckv, w: S.Workload, seed_offset: int = 0):
+        self.ckv, self.w = ckv, w
+        wseed = S.Workload(w.name, w.seq_lens, w.num_heads, w.head_dim, w.rope_dim, w.window,
+                           w.layers, w.paged, w.from_scratch, w.seed + seed_offset, w.description)
+        self.gen = S.generate(wseed, "cuda")
+        self.seq = self.gen["seq_len"]
+        self.prev = (self.seq - 1).to(torch.int32)
+        self.layers = []
+        for lay, ls in zip(self.gen["layers"], w.layers):
+            cfg = ckv.LayerConfig(w.num_heads, w.head_dim, w.rope_dim, ls.ratio, w.window,
+                                  ls.comp_dtype, ls.win_dtype)
+            cache = ckv.cache_from_tensors(cfg, w.batch, lay["comp_codes"], lay["comp_scales"],
+                                           lay["win_codes"], lay["win_scales"], lay["comp_table"],
+                                           lay["win_table"])
+            dl = ckv.DecodeLayer(cfg, cache, w.batch, max(w.seq_lens), ls.top_k)
+            cu = lay["cu_setup"]
+            n = int((cu[1:] - cu[:-1]).max().item())
+            if n > 0:  # the unfinished group before the decode token (setup, untimed)
+                dl.append(lay["setup_start"].to(torch.int32), lay["kv_setup"], lay["logit_setup"],
+                          cu_new=cu, max_new=n)
+            self.layers.append((dl, lay))
+        torch.cuda.synchronize()
+
+    def run(self, q_list=None, kv_list=None, lg_list=None, seq=None, prev=None):
+        seq = self.seq if seq is None else seq
+        prev = self.prev if prev is None else prev
+        outs = []
+        for i, (dl, lay) in enumerate(self.layers):
+            q = lay["q"] if q_list is None else q_list[i]
+            kv = lay["kv_new"] if kv_list is None else kv_list[i]
+            lg = lay["logit_new"] if lg_list is None else lg_list[i]
+            outs.append(dl.step(seq, prev, q, kv, lg))
+        return outs
+
+    def status(self) -> int:
+        return max(int(dl.status[0].item()) & 0xffffffff for dl, _ in self.layers)
+
+
+def run_cuda(args, w: S.Workload):
+    import compressed_kv_sparse_compress_b200 as ckv
+    ckv.load_library()
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    step = Step(ckv, w, seed_offset=rank)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if ws > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    dominant = "score_kernel" if any(ls.top_k is not None for ls in w.layers) else "attention_kernel"
+    prof_which = ckv.CKV_PROF_SCORE if dominant == "score_kernel" else ckv.CKV_PROF_ATTENTION
+    n_dom = sum(1 for ls in w.layers if (ls.top_k is not None) == (dominant == "score_kernel"))
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step.run()
+    barrier()
+    if step.status() != 0:
+        raise RuntimeError(f"device status {step.status():#x} after warm-up")
+
+    # ---- timed region: K steps, device events per step, dominant kernel events per launch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(n_dom)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    launches0 = ckv.launch_count()
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        if n_dom == 1:
+            ckv.profile_events(prof_which, kev[i][0][0], kev[i][0][1])
+            step.run()
+        else:  # one event pair per layer of the dominant kind
+            outs = []
+            k = 0
+            for dl, lay in step.layers:
+                is_dom = (dl.top_k is not None) == (dominant == "score_kernel")
+                if is_dom:
+                    ckv.profile_events(prof_which, kev[i][k][0], kev[i][k][1])
+                    k += 1
+                else:
+                    ckv.profile_events(prof_which)
+                outs.append(dl.step(step.seq, step.prev, lay["q"], lay["kv_new"], lay["logit_new"]))
+        ev[i][1].record(stream)
+    barrier()
+    ckv.profile_events(prof_which)
+    launches = ckv.launch_count() - launches0
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    dom_ms = [a.elapsed_time(b) for row in kev for a, b in row]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    if step.status() != 0:
+        raise RuntimeError(f"device status {step.status():#x} in the timed region")
+
+    # ---- end to end through the public API: pinned host inputs -> device -> result on host
+    q_h = [lay["q"].cpu().pin_memory() for _, lay in step.layers]
+    kv_h = [lay["kv_new"].cpu().pin_memory() for _, lay in step.layers]
+    lg_h = [lay["logit_new"].cpu().pin_memory() for _, lay in step.layers]
+    seq_h = step.seq.cpu().pin_memory()
+    out_h = [torch.empty_like(lay["q"], device="cpu").pin_memory() for _, lay in step.layers]
+    q_d = [torch.empty_like(x, device=dev) for x in q_h]
+    kv_d = [torch.empty_like(x, device=dev) for x in kv_h]
+    lg_d = [torch.empty_like(x, device=dev) for x in lg_h]
+    seq_d = torch.empty_like(seq_h, device=dev)
+    h2d = sum(x.numel() * x.element_size() for x in q_h + kv_h + lg_h) + seq_h.numel() * 4
+    d2h = sum(x.numel() * x.element_size() for x in out_h)
+
+    def e2e_step():
+        seq_d.copy_(seq_h, non_blocking=True)
+        for a, b in zip(q_d + kv_d + lg_d, q_h + kv_h + lg_h):
+            a.copy_(b, non_blocking=True)
+        prev_d = seq_d - 1
+        outs = step.run(q_d, kv_d, lg_d, seq_d, prev_d.to(torch.int32))
+        for o, oh in zip(outs, out_h):
+            oh.copy_(o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        flush.zero_()
+        e2e_step()
+    barrier()
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        eev[i][0].record(stream)
+        e2e_step()
+        eev[i][1].record(stream)
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+
+    units = w.batch * len(w.layers) * ws  # queries*layers per step over all ranks
+    value = units * args.steps / (total_ms / 1e3)
+    peak, peak_src = measured_peak()
+    lb = [layer_bytes(w, ls) for ls in w.layers]
+    if dominant == "score_kernel":
+        dom_bytes = sum(b["indexer"] for b, ls in zip(lb, w.layers) if ls.top_k is not None) / n_dom
+    else:
+        dom_bytes = sum(b["attention"] for b, ls in zip(lb, w.layers) if ls.top_k is None) / n_dom
+    dom_avg_ms = sum(dom_ms) / len(dom_ms)
+    achieved = dom_bytes / (dom_avg_ms / 1e3) / 1e9
+    step_bytes = sum(sum(b.values()) for b in lb)
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {
+            "workload": w.name, "batch_per_gpu": w.batch, "seq_lens": summarize_lens(w.seq_lens),
+            "heads": w.num_heads, "head_dim": w.head_dim, "rope_dim": w.rope_dim,
+            "window": w.window,
+            "layers": [{"ratio": ls.ratio, "top_k": ls.top_k, "comp_cache": ls.comp_dtype,
+                        "win_cache": ls.win_dtype} for ls in w.layers],
+            "paged": w.paged, "parallelism": f"dp{ws} (independent requests per GPU)",
+            "l2": "flushed before every step (256 MiB write, outside the step events)",
+            "step": "append decode token + indexer/top-k + attention (+ split combine), per layer",
+        },
+        "hbm": {"step_bytes": step_bytes,
+                "step_GBps": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
+                "frac_of_measured": step_bytes / (total_ms / args.steps / 1e3) / 1e9 / peak,
+                "frac_of_8TBps": step_bytes / (total_ms / args.steps / 1e3) / 1e9 / 8000.0},
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
+                     "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
+                     "avg_launch_us": dom_avg_ms * 1e3, "algorithmic_bytes": dom_bytes,
+                     "traffic": traffic_record(dominant, w.name)},
+        "e2e": {"value": units * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if ws > 1:
+        torch.distributed.barrier()
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, step, args.cpu_seconds)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+    return result if rank == 0 else None
+
+
+def summarize_lens(lens):
+    if len(set(lens)) == 1:
+        return lens[0]
+    return {"n": len(lens), "min": min(lens), "median": int(statistics.median(lens)), "max": max(lens),
+            "sum": sum(lens)}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle (the reported baseline, and the --impl reference arm)
+# ------------------------------------------------------------------------------------------------
+
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_request(w, gen_host, li, b, O):
+    """The oracle's whole step for request b of layer li (append + select + attention)."""
+    ls = w.layers[li]
+    lay = gen_host["layers"][li]
+    cfg = O.LayerCfg(w.num_heads, w.head_dim, w.rope_dim, ls.ratio, w.window, ls.comp_dtype,
+                     ls.win_dtype)
+    cache = O.LayerCache(lay["comp_codes"], lay["comp_scales"], lay["win_codes"], lay["win_scales"],
+                         lay["comp_table"], lay["win_table"], residue=[[] for _ in range(w.batch)])
+    L = w.seq_lens[b]
+    start = int(lay["setup_start"][b])
+    cu = lay["cu_setup"]
+    O.append_tokens(cfg, cache, b, start, lay["kv_setup"][cu[b]:cu[b + 1]], lay["logit_setup"][cu[b]:cu[b + 1]])
+    O.append_tokens(cfg, cache, b, L - 1, lay["kv_new"][b:b + 1], lay["logit_new"][b:b + 1])
+    O.decode_layer(cfg, cache, b, lay["q"][b], L, ls.top_k)
+
+
+def host_inputs(gen):
+    out = {"layers": []}
+    for lay in gen["layers"]:
+        out["layers"].append({k: (v.cpu().numpy().copy() if torch.is_tensor(v) else v)
+                              for k, v in lay.items()})
+    return out
+
+
+def cpu_baseline(w, step, seconds):
+    from oracle import ckv_oracle as O
+    gen_host = host_inputs(step.gen)
+    done = 0
+    t0 = time.perf_counter()
+    reqs = []
+    while True:
+        for li in range(len(w.layers)):
+            b = done % w.batch
+            oracle_request(w, gen_host, li, b, O)
+            reqs.append((li, b))
+        done += 1
+        if time.perf_counter() - t0 >= seconds or done >= 4 * w.batch:
+            break
+    el = time.perf_counter() - t0
+    return {"value": done * len(w.layers) / el, "unit": UNIT, "cores": oracle_threads(),
+            "kind": "oracle",
+            "sample": f"{done} requests x {len(w.layers)} layer(s) of {w.name} (same seeded inputs), "
+                      f"each a full append+select+attend in the fp64 numpy oracle; {el:.1f} s"}
+
+
+def run_reference(args, w):
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return None
+    from oracle import ckv_oracle as O
+    gen = S.generate(w, "cpu")
+    gen_host = host_inputs(gen)
+    per_step = w.batch if args.reference_requests <= 0 else min(w.batch, args.reference_requests)
+    b = 0
+    for _ in range(args.warmup):
+        for li in range(len(w.layers)):
+            oracle_request(w, gen_host, li, b % w.batch, O)
+        b += 1
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for _r in range(per_step):
+            for li in range(len(w.layers)):
+                oracle_request(w, gen_host, li, b % w.batch, O)
+            b += 1
+    el = time.perf_counter() - t0
+    units = args.steps * per_step * len(w.layers)
+    value = units / el
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "sample_requests_per_step": per_step,
+                   "note": "CPU oracle (fp64 numpy) on a bounded sample of the workload's requests"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                         "sample": f"{per_step} request(s) x {len(w.layers)} layer(s) per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(S.WORKLOADS))
+    ap.add_argument("--impl", default="ckv", choices=["ckv", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-requests", type=int, default=0,
+                    help="requests of the batch the reference arm runs per step (0: all)")
+    args = ap.parse_args()
+    w = S.WORKLOADS[args.workload]()
+    res = run_reference(args, w) if args.impl == "reference" else run_cuda(args, w)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

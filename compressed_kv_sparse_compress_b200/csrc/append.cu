@@ -1,0 +1,239 @@
+// Step 1 of the decode path: the KV compressor and cache append.
+//
+// 24-ai.news "vLLM uveo DeepSeek V4 s 8,7x manjim KV cacheom", section "Kako funkcionira
+// optimizacija KV cachea?": tokens are folded by a weighted sum (4x to 128x) and a local window
+// keeps full vectors; section "Sto je vLLM morao rijesiti u integraciji?": the compressor
+// remainder is held as sliding-window state. Readings: one scalar logit per token, softmax
+// weights within the group, each token rotated at its own position before the sum.
+//
+// One CTA works on whole groups of one request (blockIdx.y). Block x = 0 owns the first group the
+// call touches (the only one that reads the residue ring) and, after it, the trailing unfinished
+// group (the only one that writes the ring), so ring reads happen before ring writes. Every other
+// group of the call is made of new tokens only and is handled by any block, grid-strided.
+
+#include "ckv_internal.h"
+
+namespace ckv {
+namespace {
+
+constexpr int kAppendThreads = 256;
+constexpr int kMaxPairsPerThread = 2;  // D <= 1024
+
+struct AppendArgs {
+  LayerParams p;
+  const int32_t* prev_len;
+  const int32_t* cu_new;
+  int max_seq_len;
+  const float* kv_new;
+  const float* logit_new;
+  uint32_t* status;
+};
+
+__device__ float block_max(float v, float* red) {
+  v = warp_max(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float m = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
+  if (w == 0) m = warp_max(m);
+  if (threadIdx.x == 0) red[0] = m;
+  __syncthreads();
+  return red[0];
+}
+
+// rotated fp32 value of dims (2*pr, 2*pr+1) of a raw token at position pos
+__device__ __forceinline__ float2 rotate_raw_pair(const AppendArgs& a, const float* raw, int pr,
+                                                  int64_t pos) {
+  const LayerParams& p = a.p;
+  const float x0 = raw[2 * pr], x1 = raw[2 * pr + 1];
+  const int first_rope_pair = (p.D - p.d_r) / 2;
+  if (pr < first_rope_pair) return make_float2(x0, x1);
+  double o0, o1;
+  rope_rotate_pair(x0, x1, static_cast<double>(pos),
+                   rope_inv_freq(pr - first_rope_pair, p.d_r, p.rope_base), false, &o0, &o1);
+  return make_float2(static_cast<float>(o0), static_cast<float>(o1));
+}
+
+// Writes one rotated token (pairs held by this thread) into the window cache.
+__device__ void write_window_token(const AppendArgs& a, int b, int64_t pos,
+                                   const float2 (&x)[kMaxPairsPerThread], float* red) {
+  const LayerParams& p = a.p;
+  const int npairs = p.D / 2;
+  const int64_t row = win_row(p, b, pos, a.status);  // uniform across the block
+  if (p.win_dtype == CKV_F32) {
+    if (row < 0) return;
+    float2* dst = reinterpret_cast<float2*>(p.win_codes + row * p.win_row_bytes);
+    for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) dst[pr] = x[k];
+    return;
+  }
+  // FP8 e4m3 with one fp32 scale per token: s = amax / 448 (1 when the token is zero)
+  float amax = 0.f;
+  for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x)
+    amax = fmaxf(amax, fmaxf(fabsf(x[k].x), fabsf(x[k].y)));
+  amax = block_max(amax, red);
+  if (row < 0) return;
+  const float s = amax > 0.f ? amax / 448.0f : 1.0f;
+  uint16_t* dst = reinterpret_cast<uint16_t*>(p.win_codes + row * p.win_row_bytes);
+  for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) {
+    const uint32_t c0 = f32_to_e4m3_satfinite(x[k].x / s);
+    const uint32_t c1 = f32_to_e4m3_satfinite(x[k].y / s);
+    dst[pr] = static_cast<uint16_t>(c0 | (c1 << 8));
+  }
+  if (threadIdx.x == 0) p.win_scales[row] = s;
+}
+
+// Quantises entry c (fp32 in shared memory) into compressed pool row `row`.
+__device__ void store_entry(const LayerParams& p, int64_t row, const float* c) {
+  const int D = p.D;
+  uint8_t* dst = p.comp_codes + row * p.comp_row_bytes;
+  if (p.comp_dtype == CKV_F32) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) reinterpret_cast<float*>(dst)[d] = c[d];
+  } else if (p.comp_dtype == CKV_BF16) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x)
+      reinterpret_cast<uint16_t*>(dst)[d] = f32_to_bf16_rne(c[d]);
+  } else {  // NVFP4: per 16 elements scale = e4m3(amax / 6), codes = e2m1(x / scale)
+    uint8_t* sdst = p.comp_scales + row * (D / 16);
+    for (int blk = threadIdx.x; blk < D / 16; blk += blockDim.x) {
+      const float* v = c + 16 * blk;
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+      const uint8_t sc = f32_to_e4m3_satfinite(amax / 6.0f);
+      const float s = e4m3_to_f32(sc);
+      uint32_t lo = 0, hi = 0;
+      if (s > 0.f) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) lo |= static_cast<uint32_t>(f32_to_e2m1_satfinite(v[e] / s)) << (4 * e);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) hi |= static_cast<uint32_t>(f32_to_e2m1_satfinite(v[8 + e] / s)) << (4 * e);
+      }
+      reinterpret_cast<uint2*>(dst)[blk] = make_uint2(lo, hi);
+      sdst[blk] = sc;
+    }
+  }
+}
+
+// Handles group g of request b: writes the new tokens' window / ring slots and, when the group
+// is complete, folds it into entry g.
+__device__ void process_group(const AppendArgs& a, int b, int64_t g, int64_t prev, int64_t new_len,
+                              int64_t row0, float* smem) {
+  const LayerParams& p = a.p;
+  const int r = p.r, D = p.D, npairs = D / 2;
+  float* w = smem;            // [r] weights
+  float* c = smem + 256;      // [D] entry
+  float* red = c + 1024;      // [32] reductions
+  const int64_t t0 = g * r;
+  const int64_t t_end = min(t0 + r, new_len);
+  const bool complete = (t0 + r) <= new_len;
+  float* ring = p.res_kv + static_cast<int64_t>(b) * r * D;
+  float* ring_logit = p.res_logit + static_cast<int64_t>(b) * r;
+
+  // new tokens of the group: window and (unfinished group) residue ring
+  for (int64_t pos = max(t0, prev); pos < t_end; ++pos) {
+    const bool to_window = p.W > 0 && pos >= new_len - p.W;
+    if (!to_window && complete) continue;
+    const float* raw = a.kv_new + (row0 + (pos - prev)) * D;
+    float2 x[kMaxPairsPerThread];
+    for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) x[k] = rotate_raw_pair(a, raw, pr, pos);
+    if (!complete) {
+      float2* dst = reinterpret_cast<float2*>(ring + (pos % r) * D);
+      for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) dst[pr] = x[k];
+      if (threadIdx.x == 0) ring_logit[pos % r] = a.logit_new[row0 + (pos - prev)];
+    }
+    if (to_window) write_window_token(a, b, pos, x, red);
+  }
+  if (!complete) return;
+
+  // softmax of the group's logits (positions before prev come from the ring)
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float m = -INFINITY;
+    for (int t = threadIdx.x; t < r; t += 32) {
+      const int64_t pos = t0 + t;
+      const float lg = pos < prev ? ring_logit[pos % r] : a.logit_new[row0 + (pos - prev)];
+      w[t] = lg;
+      m = fmaxf(m, lg);
+    }
+    m = warp_max(m);
+    float s = 0.f;
+    for (int t = threadIdx.x; t < r; t += 32) {
+      const float e = expf(w[t] - m);
+      w[t] = e;
+      s += e;
+    }
+    s = warp_sum(s);
+    for (int t = threadIdx.x; t < r; t += 32) w[t] = w[t] / s;
+  }
+  __syncthreads();
+  // entry = sum over the group's tokens, in token order, of w_t * rotated token t
+  for (int pr = threadIdx.x; pr < npairs; pr += blockDim.x) {
+    float2 acc = make_float2(0.f, 0.f);
+    for (int t = 0; t < r; ++t) {
+      const int64_t pos = t0 + t;
+      float2 x;
+      if (pos < prev) {
+        x = reinterpret_cast<const float2*>(ring + (pos % r) * D)[pr];
+      } else {
+        x = rotate_raw_pair(a, a.kv_new + (row0 + (pos - prev)) * D, pr, pos);
+      }
+      acc.x = fmaf(w[t], x.x, acc.x);
+      acc.y = fmaf(w[t], x.y, acc.y);
+    }
+    c[2 * pr] = acc.x;
+    c[2 * pr + 1] = acc.y;
+  }
+  __syncthreads();
+  const int64_t row = comp_row(p, b, g, a.status);
+  if (row >= 0) store_entry(p, row, c);
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
+  __shared__ float smem[256 + 1024 + 32];
+  const int b = blockIdx.y;
+  const int64_t prev = a.prev_len[b];
+  int64_t row0, n;
+  if (a.cu_new) {
+    row0 = a.cu_new[b];
+    n = static_cast<int64_t>(a.cu_new[b + 1]) - row0;
+  } else {
+    row0 = b;
+    n = 1;
+  }
+  if (n <= 0) return;
+  if (prev < 0 || prev + n > a.max_seq_len) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(a.status, CKV_DEV_BAD_LENGTH);
+    return;
+  }
+  const int r = a.p.r;
+  const int64_t new_len = prev + n;
+  const int64_t gA = prev / r, gB = (new_len - 1) / r;
+  const bool trailing_unfinished = (new_len % r) != 0;
+  if (blockIdx.x == 0) {
+    process_group(a, b, gA, prev, new_len, row0, smem);
+    __syncthreads();
+    if (gB != gA && trailing_unfinished) process_group(a, b, gB, prev, new_len, row0, smem);
+  }
+  const int64_t mid_end = trailing_unfinished ? gB : gB + 1;
+  for (int64_t g = gA + 1 + blockIdx.x; g < mid_end; g += gridDim.x) {
+    __syncthreads();
+    process_group(a, b, g, prev, new_len, row0, smem);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_len,
+                          const int32_t* cu_new, int max_new, int max_seq_len, const float* kv_new,
+                          const float* logit_new, uint32_t* status, cudaStream_t stream) {
+  AppendArgs a{p, prev_len, cu_new, max_seq_len, kv_new, logit_new, status};
+  const int64_t groups = static_cast<int64_t>(max_new) / p.r + 2;
+  const int gx = static_cast<int>(groups < 512 ? groups : 512);
+  dim3 grid(gx, batch);
+  append_kernel<<<grid, kAppendThreads, 0, stream>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace ckv

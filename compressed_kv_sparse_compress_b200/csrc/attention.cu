@@ -1,0 +1,269 @@
+// Step 3 of the decode path: joint attention over the selected compressed entries and the
+// sliding window, with one shared K=V vector per key and inverse RoPE on the output.
+//
+// 24-ai.news "vLLM uveo DeepSeek V4 s 8,7x manjim KV cacheom", section "Kako funkcionira
+// optimizacija KV cachea?": shared K=V vectors with inverse RoPE, sparse attention over the
+// top-k compressed tokens, a local window of full vectors. Reading: one softmax over the union
+// of the selected entries and the window tokens [max(0, L-W), L), without de-duplication.
+//
+// The key list of request b is: selected entries (or all floor(L/r) for a dense layer), then the
+// window tokens. It is cut into splits of keys_per_split keys; each split writes an
+// un-normalised partial (running max m, sum l, sum of p*x) per head, and attn_combine merges
+// the splits by log-sum-exp, normalises, and rotates the rotary dims back by -(L-1).
+//
+// This file holds the CUDA-core path (any head count, fp32 accumulation of everything) and the
+// combine. The tensor-core path for H=64 lives in attention_tc.cu and writes the same partials.
+
+#include "ckv_internal.h"
+
+namespace ckv {
+
+bool attention_tc_supported(const LayerParams& p);
+int attention_tc_keys_per_split();
+cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,
+                                int max_seq_len, const float* q, const int32_t* idx,
+                                const int32_t* cnt, int idx_stride, const AttnWs& ws,
+                                uint32_t* status, cudaStream_t stream);
+
+namespace {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSimtKeys = 32;  // keys per split of the CUDA-core path
+constexpr int kCombineThreads = 128;
+
+struct KeyList {
+  int64_t n_c, n_sel, n_win, n_keys;
+};
+
+__device__ __forceinline__ KeyList key_list(const LayerParams& p, int L, const int32_t* cnt,
+                                            bool sparse, int idx_stride, int b) {
+  KeyList k;
+  k.n_c = L / p.r;
+  k.n_sel = sparse ? min(static_cast<int64_t>(max(cnt[b], 0)), static_cast<int64_t>(idx_stride)) : k.n_c;
+  k.n_win = min(p.W, L);
+  k.n_keys = k.n_sel + k.n_win;
+  return k;
+}
+
+// Decodes pair pr (dims 2pr, 2pr+1) of compressed row `row`.
+__device__ __forceinline__ float2 comp_pair(const LayerParams& p, int64_t row, int pr) {
+  const uint8_t* base = p.comp_codes + row * p.comp_row_bytes;
+  if (p.comp_dtype == CKV_F32) return reinterpret_cast<const float2*>(base)[pr];
+  if (p.comp_dtype == CKV_BF16) {
+    const uint32_t w = reinterpret_cast<const uint32_t*>(base)[pr];
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  }
+  const float s = e4m3_to_f32(p.comp_scales[row * (p.D / 16) + pr / 8]);
+  const float2 v = __half22float2(e2m1x2_to_half2(base[pr]));
+  return make_float2(v.x * s, v.y * s);
+}
+
+__device__ __forceinline__ float2 win_pair(const LayerParams& p, int64_t row, int pr) {
+  const uint8_t* base = p.win_codes + row * p.win_row_bytes;
+  if (p.win_dtype == CKV_F32) return reinterpret_cast<const float2*>(base)[pr];
+  const uint16_t c = reinterpret_cast<const uint16_t*>(base)[pr];
+  const float s = p.win_scales[row];
+  return make_float2(e4m3_to_f32(c & 0xff) * s, e4m3_to_f32(c >> 8) * s);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
+    LayerParams p, const int32_t* seq_len, int max_seq_len, const float* q, const int32_t* idx,
+    const int32_t* cnt, int idx_stride, AttnWs ws, uint32_t* status) {
+  constexpr int NPL = D / 64;  // rotary-aligned pairs per lane
+  extern __shared__ float xs[];  // [kSimtKeys][D]
+  __shared__ int valid[kSimtKeys];
+  const int b = blockIdx.y, s = blockIdx.x;
+  const int L = seq_len[b];
+  if (L < 1 || L > max_seq_len) return;  // flagged by the combine
+  const KeyList kl = key_list(p, L, cnt, idx != nullptr, idx_stride, b);
+  const int64_t k0 = static_cast<int64_t>(s) * kSimtKeys;
+  if (k0 >= kl.n_keys) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  for (int i = warp; i < kSimtKeys; i += kSimtThreads / 32) {
+    const int64_t kk = k0 + i;
+    bool ok = kk < kl.n_keys;
+    int64_t row = -1;
+    bool is_win = false;
+    if (ok && kk < kl.n_sel) {
+      const int64_t ent = idx ? idx[static_cast<int64_t>(b) * idx_stride + kk] : kk;
+      if (ent < 0 || ent >= kl.n_c) {
+        if (lane == 0) atomicOr(status, CKV_DEV_BAD_INDEX);
+        ok = false;
+      } else {
+        row = comp_row(p, b, ent, status);
+      }
+    } else if (ok) {
+      is_win = true;
+      row = win_row(p, b, L - kl.n_win + (kk - kl.n_sel), status);
+    }
+    ok = ok && row >= 0;
+    if (ok) {
+      for (int pr = lane; pr < D / 2; pr += 32)
+        reinterpret_cast<float2*>(xs + i * D)[pr] = is_win ? win_pair(p, row, pr) : comp_pair(p, row, pr);
+    }
+    if (lane == 0) valid[i] = ok;
+  }
+  __syncthreads();
+
+  const int first_rope = (D - p.d_r) / 2;
+  const double pos = static_cast<double>(L - 1);
+  for (int h = warp; h < p.H; h += kSimtThreads / 32) {
+    const float* qh = q + (static_cast<int64_t>(b) * p.H + h) * D;
+    float2 qv[NPL], ov[NPL];
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+      const int pr = lane + 32 * k;
+      float2 v = reinterpret_cast<const float2*>(qh)[pr];
+      if (pr >= first_rope) {
+        double a, c;
+        rope_rotate_pair(v.x, v.y, pos, rope_inv_freq(pr - first_rope, p.d_r, p.rope_base), false, &a, &c);
+        v = make_float2(static_cast<float>(a), static_cast<float>(c));
+      }
+      qv[k] = v;
+      ov[k] = make_float2(0.f, 0.f);
+    }
+    float m = -INFINITY, l = 0.f;
+    for (int i = 0; i < kSimtKeys; ++i) {
+      if (!valid[i]) continue;
+      const float2* x = reinterpret_cast<const float2*>(xs + i * D);
+      float dot = 0.f;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        const float2 xv = x[lane + 32 * k];
+        dot = fmaf(qv[k].x, xv.x, dot);
+        dot = fmaf(qv[k].y, xv.y, dot);
+      }
+      dot = warp_sum(dot) * p.sm_scale;
+      const float m_new = fmaxf(m, dot);
+      const float alpha = expf(m - m_new);
+      const float pj = expf(dot - m_new);
+      l = l * alpha + pj;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        const float2 xv = x[lane + 32 * k];
+        ov[k].x = fmaf(pj, xv.x, ov[k].x * alpha);
+        ov[k].y = fmaf(pj, xv.y, ov[k].y * alpha);
+      }
+      m = m_new;
+    }
+    const int64_t slot = (static_cast<int64_t>(b) * ws.splits + s) * p.H + h;
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) reinterpret_cast<float2*>(ws.part_o + slot * D)[lane + 32 * k] = ov[k];
+    if (lane == 0) reinterpret_cast<float2*>(ws.part_ml)[slot] = make_float2(m, l);
+  }
+}
+
+__global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(
+    LayerParams p, const int32_t* seq_len, int max_seq_len, const int32_t* cnt, bool sparse,
+    int idx_stride, AttnWs ws, float* out, uint32_t* status) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int D = p.D;
+  float* o = out + (static_cast<int64_t>(b) * p.H + h) * D;
+  const int L = seq_len[b];
+  if (L < 1 || L > max_seq_len) {
+    if (h == 0 && threadIdx.x == 0) atomicOr(status, CKV_DEV_BAD_LENGTH);
+    for (int d = threadIdx.x; d < D; d += blockDim.x) o[d] = 0.f;
+    return;
+  }
+  const KeyList kl = key_list(p, L, cnt, sparse, idx_stride, b);
+  const int ns = static_cast<int>((kl.n_keys + ws.keys_per_split - 1) / ws.keys_per_split);
+  const float2* ml = reinterpret_cast<const float2*>(ws.part_ml);
+  const int64_t base = static_cast<int64_t>(b) * ws.splits;
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) {
+    const float2 v = ml[(base + s) * p.H + h];
+    if (v.y > 0.f) M = fmaxf(M, v.x);
+  }
+  float Z = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const float2 v = ml[(base + s) * p.H + h];
+    if (v.y > 0.f) Z += v.y * expf(v.x - M);
+  }
+  const float inv = Z > 0.f ? 1.f / Z : 0.f;
+  const int first_rope = (D - p.d_r) / 2;
+  for (int pr = threadIdx.x; pr < D / 2; pr += blockDim.x) {
+    float2 acc = make_float2(0.f, 0.f);
+    for (int s = 0; s < ns; ++s) {
+      const float2 v = ml[(base + s) * p.H + h];
+      if (!(v.y > 0.f)) continue;
+      const float w = expf(v.x - M);
+      const float2 x = reinterpret_cast<const float2*>(ws.part_o + ((base + s) * p.H + h) * D)[pr];
+      acc.x = fmaf(w, x.x, acc.x);
+      acc.y = fmaf(w, x.y, acc.y);
+    }
+    acc.x *= inv;
+    acc.y *= inv;
+    if (pr >= first_rope) {
+      double a, c;
+      rope_rotate_pair(acc.x, acc.y, static_cast<double>(L - 1),
+                       rope_inv_freq(pr - first_rope, p.d_r, p.rope_base), true, &a, &c);
+      acc = make_float2(static_cast<float>(a), static_cast<float>(c));
+    }
+    reinterpret_cast<float2*>(o)[pr] = acc;
+  }
+}
+
+template <int D>
+cudaError_t launch_simt_d(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
+                          const float* q, const int32_t* idx, const int32_t* cnt, int idx_stride,
+                          const AttnWs& ws, uint32_t* status, cudaStream_t stream) {
+  const int smem = kSimtKeys * D * static_cast<int>(sizeof(float));
+  auto kern = attn_simt_kernel<D>;
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(ws.splits, batch);
+  kern<<<grid, kSimtThreads, smem, stream>>>(p, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len,
+                           int max_selected) {
+  AttnWs w{};
+  const int64_t sel = max_selected > 0 ? max_selected : static_cast<int64_t>(max_seq_len) / p.r;
+  const int64_t keys = sel + (p.W < max_seq_len ? p.W : max_seq_len);
+  w.keys_per_split = attention_tc_supported(p) ? attention_tc_keys_per_split() : kSimtKeys;
+  w.splits = static_cast<int>(keys > 0 ? (keys + w.keys_per_split - 1) / w.keys_per_split : 1);
+  const size_t n_slot = static_cast<size_t>(batch) * w.splits * p.H;
+  const size_t o_bytes = align_up(n_slot * p.D * sizeof(float), 256);
+  const size_t ml_bytes = align_up(n_slot * 2 * sizeof(float), 256);
+  if (base) {
+    w.part_o = static_cast<float*>(base);
+    w.part_ml = reinterpret_cast<float*>(static_cast<char*>(base) + o_bytes);
+  }
+  w.bytes = o_bytes + ml_bytes;
+  return w;
+}
+
+cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq_len,
+                             int max_seq_len, const float* q, const int32_t* idx,
+                             const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
+                             uint32_t* status, cudaStream_t stream) {
+  cudaError_t e;
+  prof_begin(kProfAttention, stream);
+  if (attention_tc_supported(p)) {
+    e = launch_attention_tc(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);
+  } else {
+    switch (p.D) {
+      case 64: e = launch_simt_d<64>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream); break;
+      case 128: e = launch_simt_d<128>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream); break;
+      case 256: e = launch_simt_d<256>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream); break;
+      case 512: e = launch_simt_d<512>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream); break;
+      case 1024: e = launch_simt_d<1024>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream); break;
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  prof_end(kProfAttention, stream);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.H, batch);
+  attn_combine_kernel<<<grid, kCombineThreads, 0, stream>>>(p, seq_len, max_seq_len, cnt, idx != nullptr,
+                                                           idx_stride, ws, out, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace ckv

@@ -1,0 +1,316 @@
+// The C ABI of libckv (include/ckv.h): argument validation, block pools, workspace carving and
+// dispatch to the kernels. Host code only; nothing here touches device memory directly.
+
+#include <atomic>
+#include <cmath>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "ckv_internal.h"
+
+namespace ckv {
+
+static std::atomic<uint64_t> g_launches{0};
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static cudaEvent_t g_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+
+void prof_begin(ProfPoint which, cudaStream_t stream) {
+  if (g_prof[which][0]) cudaEventRecord(g_prof[which][0], stream);
+}
+
+void prof_end(ProfPoint which, cudaStream_t stream) {
+  if (g_prof[which][1]) cudaEventRecord(g_prof[which][1], stream);
+}
+
+int sm_count() {
+  static int cache[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+cudaError_t allow_smem(const void* kernel, int bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int row_bytes_comp(int dtype, int D) {
+  switch (dtype) {
+    case CKV_F32: return 4 * D;
+    case CKV_BF16: return 2 * D;
+    case CKV_NVFP4: return D / 2;
+    default: return -1;
+  }
+}
+
+int row_bytes_win(int dtype, int D) {
+  switch (dtype) {
+    case CKV_F32: return 4 * D;
+    case CKV_FP8_E4M3: return D;
+    default: return -1;
+  }
+}
+
+int check_cfg(const ckv_layer_cfg* c) {
+  if (!c) return CKV_ERR_INVALID_ARG;
+  if (c->num_heads < 1 || c->num_heads > 1024) return CKV_ERR_INVALID_ARG;
+  if (c->ratio < 1 || c->ratio > 256 || !is_pow2(c->ratio)) return CKV_ERR_INVALID_ARG;
+  if (c->window < 0 || c->window > 256) return CKV_ERR_INVALID_ARG;
+  if (c->rope_dim < 0 || c->rope_dim > c->head_dim || (c->rope_dim & 1)) return CKV_ERR_INVALID_ARG;
+  if (!(c->sm_scale >= 0.f) || !std::isfinite(c->sm_scale)) return CKV_ERR_INVALID_ARG;
+  if (!(c->rope_base >= 0.f) || !std::isfinite(c->rope_base)) return CKV_ERR_INVALID_ARG;
+  if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256 && c->head_dim != 512 &&
+      c->head_dim != 1024)
+    return CKV_ERR_UNSUPPORTED;
+  if (row_bytes_comp(c->comp_dtype, c->head_dim) < 0) return CKV_ERR_UNSUPPORTED;
+  if (row_bytes_win(c->win_dtype, c->head_dim) < 0) return CKV_ERR_UNSUPPORTED;
+  return CKV_OK;
+}
+
+// Validates cfg + cache and fills the kernel parameter block. need_residue: the append path.
+int make_params(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int batch, int max_seq_len,
+                bool need_residue, LayerParams* p) {
+  int st = check_cfg(cfg);
+  if (st != CKV_OK) return st;
+  if (!cache || batch < 1 || max_seq_len < 1) return CKV_ERR_INVALID_ARG;
+  const int D = cfg->head_dim;
+  if (!cache->comp_codes || !aligned16(cache->comp_codes)) return CKV_ERR_INVALID_ARG;
+  if (cfg->comp_dtype == CKV_NVFP4 && (!cache->comp_scales || !aligned16(cache->comp_scales)))
+    return CKV_ERR_INVALID_ARG;
+  if (cfg->window > 0) {
+    if (!cache->win_codes || !aligned16(cache->win_codes) || !cache->win_table ||
+        !aligned16(cache->win_table) || cache->win_blocks < 1)
+      return CKV_ERR_INVALID_ARG;
+    if (cfg->win_dtype == CKV_FP8_E4M3 && (!cache->win_scales || !aligned16(cache->win_scales)))
+      return CKV_ERR_INVALID_ARG;
+  }
+  if (!cache->comp_table || !aligned16(cache->comp_table) || cache->comp_blocks < 1)
+    return CKV_ERR_INVALID_ARG;
+  if (cache->table_stride < (static_cast<int64_t>(max_seq_len) + kBlockTokens - 1) / kBlockTokens)
+    return CKV_ERR_INVALID_ARG;
+  if (need_residue && (!cache->residue_kv || !aligned16(cache->residue_kv) || !cache->residue_logit ||
+                       !aligned16(cache->residue_logit)))
+    return CKV_ERR_INVALID_ARG;
+  LayerParams& q = *p;
+  q.H = cfg->num_heads;
+  q.D = D;
+  q.d_r = cfg->rope_dim;
+  q.r = cfg->ratio;
+  q.W = cfg->window;
+  q.comp_dtype = cfg->comp_dtype;
+  q.win_dtype = cfg->win_dtype;
+  q.epb = kBlockTokens / cfg->ratio;
+  q.comp_row_bytes = row_bytes_comp(cfg->comp_dtype, D);
+  q.win_row_bytes = row_bytes_win(cfg->win_dtype, D);
+  q.sm_scale = cfg->sm_scale > 0.f ? cfg->sm_scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  q.rope_base = cfg->rope_base > 0.f ? static_cast<double>(cfg->rope_base) : 10000.0;
+  q.comp_codes = static_cast<uint8_t*>(cache->comp_codes);
+  q.comp_scales = static_cast<uint8_t*>(cache->comp_scales);
+  q.win_codes = static_cast<uint8_t*>(cache->win_codes);
+  q.win_scales = cache->win_scales;
+  q.res_kv = cache->residue_kv;
+  q.res_logit = cache->residue_logit;
+  q.comp_table = cache->comp_table;
+  q.win_table = cache->win_table;
+  q.table_stride = cache->table_stride;
+  q.comp_blocks = cache->comp_blocks;
+  q.win_blocks = cfg->window > 0 ? cache->win_blocks : 0;
+  return CKV_OK;
+}
+
+}  // namespace
+}  // namespace ckv
+
+using namespace ckv;
+
+struct ckv_pool {
+  std::vector<int32_t> stack;    // free ids, top at the back
+  std::vector<uint8_t> is_free;  // per id
+};
+
+extern "C" {
+
+int kv_block_pool_create(int32_t num_blocks, ckv_pool** out) {
+  if (!out || num_blocks < 1) return CKV_ERR_INVALID_ARG;
+  ckv_pool* p = new (std::nothrow) ckv_pool;
+  if (!p) return CKV_ERR_INVALID_ARG;
+  p->stack.resize(num_blocks);
+  for (int32_t i = 0; i < num_blocks; ++i) p->stack[i] = num_blocks - 1 - i;
+  p->is_free.assign(num_blocks, 1);
+  *out = p;
+  return CKV_OK;
+}
+
+int kv_block_pool_destroy(ckv_pool* pool) {
+  delete pool;
+  return CKV_OK;
+}
+
+int kv_block_alloc(ckv_pool* pool, int32_t n, int32_t* out_ids) {
+  if (!pool || n < 0 || (n > 0 && !out_ids)) return CKV_ERR_INVALID_ARG;
+  if (static_cast<size_t>(n) > pool->stack.size()) return CKV_ERR_OUT_OF_BLOCKS;
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t id = pool->stack.back();
+    pool->stack.pop_back();
+    pool->is_free[id] = 0;
+    out_ids[i] = id;
+  }
+  return CKV_OK;
+}
+
+int kv_block_free(ckv_pool* pool, const int32_t* ids, int32_t n) {
+  if (!pool || n < 0 || (n > 0 && !ids)) return CKV_ERR_INVALID_ARG;
+  const int32_t nb = static_cast<int32_t>(pool->is_free.size());
+  // validate everything first, so a bad call frees nothing
+  std::vector<uint8_t> seen;
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t id = ids[i];
+    if (id < 0 || id >= nb || pool->is_free[id]) return CKV_ERR_INVALID_ARG;
+  }
+  seen.assign(nb, 0);
+  for (int32_t i = 0; i < n; ++i) {
+    if (seen[ids[i]]) return CKV_ERR_INVALID_ARG;
+    seen[ids[i]] = 1;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    pool->is_free[ids[i]] = 1;
+    pool->stack.push_back(ids[i]);
+  }
+  return CKV_OK;
+}
+
+int32_t kv_block_pool_num_free(const ckv_pool* pool) {
+  if (!pool) return CKV_ERR_INVALID_ARG;
+  return static_cast<int32_t>(pool->stack.size());
+}
+
+int ckv_cache_row_bytes(const ckv_layer_cfg* cfg, size_t* comp_code_bytes, size_t* comp_scale_bytes,
+                        size_t* win_code_bytes, size_t* win_scale_bytes) {
+  const int st = check_cfg(cfg);
+  if (st != CKV_OK) return st;
+  const int D = cfg->head_dim;
+  if (comp_code_bytes) *comp_code_bytes = static_cast<size_t>(row_bytes_comp(cfg->comp_dtype, D));
+  if (comp_scale_bytes) *comp_scale_bytes = cfg->comp_dtype == CKV_NVFP4 ? static_cast<size_t>(D / 16) : 0;
+  if (win_code_bytes) *win_code_bytes = static_cast<size_t>(row_bytes_win(cfg->win_dtype, D));
+  if (win_scale_bytes) *win_scale_bytes = cfg->win_dtype == CKV_FP8_E4M3 ? sizeof(float) : 0;
+  return CKV_OK;
+}
+
+int64_t ckv_score_stride(const ckv_layer_cfg* cfg, int32_t max_seq_len) {
+  if (check_cfg(cfg) != CKV_OK || max_seq_len < 1) return 0;
+  return score_stride(cfg->ratio, max_seq_len);
+}
+
+size_t ckv_indexer_workspace_bytes(const ckv_layer_cfg* cfg, int32_t batch, int32_t max_seq_len,
+                                   int32_t top_k) {
+  if (check_cfg(cfg) != CKV_OK || batch < 1 || max_seq_len < 1 || top_k < 1) return 0;
+  LayerParams p{};
+  p.D = cfg->head_dim;
+  p.r = cfg->ratio;
+  return indexer_ws_layout(nullptr, p, batch, max_seq_len).bytes;
+}
+
+size_t ckv_attention_workspace_bytes(const ckv_layer_cfg* cfg, int32_t batch, int32_t max_seq_len,
+                                     int32_t max_selected) {
+  if (check_cfg(cfg) != CKV_OK || batch < 1 || max_seq_len < 1 || max_selected < 0) return 0;
+  LayerParams p{};
+  p.H = cfg->num_heads;
+  p.D = cfg->head_dim;
+  p.r = cfg->ratio;
+  p.W = cfg->window;
+  p.comp_dtype = cfg->comp_dtype;
+  p.win_dtype = cfg->win_dtype;
+  p.d_r = cfg->rope_dim;
+  return attention_ws_layout(nullptr, p, batch, max_seq_len, max_selected).bytes;
+}
+
+int kv_compress_append(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int32_t batch,
+                       const int32_t* d_prev_len, const int32_t* d_cu_new, int32_t max_new,
+                       int32_t max_seq_len, const float* d_kv_new, const float* d_logit_new,
+                       uint32_t* d_status, void* stream) {
+  LayerParams p{};
+  const int st = make_params(cfg, cache, batch, max_seq_len, true, &p);
+  if (st != CKV_OK) return st;
+  if (!d_prev_len || !d_kv_new || !d_logit_new || !d_status || !aligned16(d_kv_new)) return CKV_ERR_INVALID_ARG;
+  if (d_cu_new ? max_new < 1 : max_new != 1) return CKV_ERR_INVALID_ARG;
+  cudaError_t e = launch_append(p, batch, d_prev_len, d_cu_new, max_new, max_seq_len, d_kv_new,
+                                d_logit_new, d_status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+}
+
+int sparse_indexer_topk(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int32_t batch,
+                        const int32_t* d_seq_len, int32_t max_seq_len, const float* d_q,
+                        int32_t top_k, int32_t* d_idx, int32_t* d_cnt, float* d_scores,
+                        void* d_ws, size_t ws_bytes, uint32_t* d_status, void* stream) {
+  LayerParams p{};
+  const int st = make_params(cfg, cache, batch, max_seq_len, false, &p);
+  if (st != CKV_OK) return st;
+  if (batch > 16384) return CKV_ERR_UNSUPPORTED;
+  if (!d_seq_len || !d_q || !d_idx || !d_cnt || !d_status || top_k < 1 || !aligned16(d_q) ||
+      !aligned16(d_idx) || !aligned16(d_cnt) || (d_scores && !aligned16(d_scores)))
+    return CKV_ERR_INVALID_ARG;
+  if (!d_ws || !aligned16(d_ws)) return CKV_ERR_WORKSPACE;
+  IndexerWs ws = indexer_ws_layout(d_ws, p, batch, max_seq_len);
+  if (ws_bytes < ws.bytes) return CKV_ERR_WORKSPACE;
+  cudaError_t e = launch_indexer(p, batch, d_seq_len, max_seq_len, d_q, top_k, d_idx, d_cnt, d_scores,
+                                 ws, d_status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+}
+
+int compressed_window_attention(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache,
+                                int32_t batch, const int32_t* d_seq_len, int32_t max_seq_len,
+                                const float* d_q, const int32_t* d_idx, const int32_t* d_cnt,
+                                int32_t idx_stride, float* d_out, void* d_ws, size_t ws_bytes,
+                                uint32_t* d_status, void* stream) {
+  LayerParams p{};
+  const int st = make_params(cfg, cache, batch, max_seq_len, false, &p);
+  if (st != CKV_OK) return st;
+  if (!d_seq_len || !d_q || !d_out || !d_status || !aligned16(d_q) || !aligned16(d_out))
+    return CKV_ERR_INVALID_ARG;
+  if (d_idx && (!d_cnt || idx_stride < 1)) return CKV_ERR_INVALID_ARG;
+  if (!d_ws || !aligned16(d_ws)) return CKV_ERR_WORKSPACE;
+  AttnWs ws = attention_ws_layout(d_ws, p, batch, max_seq_len, d_idx ? idx_stride : 0);
+  if (ws_bytes < ws.bytes) return CKV_ERR_WORKSPACE;
+  cudaError_t e = launch_attention(p, batch, d_seq_len, max_seq_len, d_q, d_idx, d_cnt,
+                                   d_idx ? idx_stride : 0, d_out, ws, d_status,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+}
+
+const char* ckv_status_str(int status) {
+  switch (status) {
+    case CKV_OK: return "ok";
+    case CKV_ERR_INVALID_ARG: return "invalid argument";
+    case CKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case CKV_ERR_OUT_OF_BLOCKS: return "block pool exhausted";
+    case CKV_ERR_WORKSPACE: return "workspace too small";
+    case CKV_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+uint64_t ckv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ckv_profile_events(int which, void* ev_begin, void* ev_end) {
+  if (which != CKV_PROF_SCORE && which != CKV_PROF_ATTENTION) return CKV_ERR_INVALID_ARG;
+  if ((ev_begin == nullptr) != (ev_end == nullptr)) return CKV_ERR_INVALID_ARG;
+  g_prof[which][0] = static_cast<cudaEvent_t>(ev_begin);
+  g_prof[which][1] = static_cast<cudaEvent_t>(ev_end);
+  return CKV_OK;
+}
+
+}  // extern "C"

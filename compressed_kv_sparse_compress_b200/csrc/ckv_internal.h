@@ -1,0 +1,69 @@
+// Internal launch interface between the C ABI layer (capi.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ckv_common.cuh"
+
+namespace ckv {
+
+// Bookkeeping of kernel launches (ckv_launch_count).
+void note_launch();
+// Multiprocessor count of the current device (cached per device).
+int sm_count();
+// Opt a kernel into more than 48 KB of dynamic shared memory on the current device, once.
+cudaError_t allow_smem(const void* kernel, int bytes);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Diagnostic events around one kernel (ckv_profile_events); no-ops when unset.
+enum ProfPoint { kProfScore = 0, kProfAttention = 1 };
+void prof_begin(ProfPoint which, cudaStream_t stream);
+void prof_end(ProfPoint which, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------- append
+cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_len,
+                          const int32_t* cu_new, int max_new, int max_seq_len, const float* kv_new,
+                          const float* logit_new, uint32_t* status, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------- indexer
+constexpr int kHistBins = 2048;  // first radix digit: the top 11 bits of the order key
+
+// Carve-up of the indexer workspace.
+struct IndexerWs {
+  float* qbar;        // [B][D]   scaled, rotated, head-averaged query
+  int32_t* n_c;       // [B]      candidate count (0 for an invalid length)
+  uint32_t* hist;     // [B][2048]
+  uint32_t* cand_cnt; // [B]
+  uint32_t* bitmap;   // [B][stride/32]
+  uint2* cand;        // [B][stride]  (order key, index) of boundary-bin candidates
+  float* scores;      // [B][stride]  when the caller passes no score buffer
+  size_t bytes;
+};
+int64_t score_stride(int ratio, int max_seq_len);
+IndexerWs indexer_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len);
+
+cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
+                           int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
+                           float* scores, const IndexerWs& ws, uint32_t* status,
+                           cudaStream_t stream);
+
+// ---------------------------------------------------------------------------- attention
+struct AttnWs {
+  float* part_o;   // [B][S][H][D]   un-normalised partial outputs
+  float* part_ml;  // [B][S][H][2]   running max and sum of each split
+  int splits;      // S: splits per request
+  int keys_per_split;
+  size_t bytes;
+};
+AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len,
+                           int max_selected);
+
+cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq_len,
+                             int max_seq_len, const float* q, const int32_t* idx,
+                             const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
+                             uint32_t* status, cudaStream_t stream);
+
+}  // namespace ckv

@@ -1,0 +1,528 @@
+// Step 2 of the decode path: the sparse MQA indexer and top-k selection.
+//
+// 24-ai.news "vLLM uveo DeepSeek V4 s 8,7x manjim KV cacheom", section "Kako funkcionira
+// optimizacija KV cachea?": attention is restricted to the top-k compressed tokens;
+// aidevelopers.cz "DeepSeek-V4.1-Flash ve vLLM", section "Vykon neprinesl jeden kernel": the
+// "Sparse MQA logits" kernel scores only the candidate positions. Reading: the score of entry j is
+// the head-average of the MQA logits, s_j = sm_scale/H * sum_h q~_h . k_j. All heads share k_j,
+// so the sum over heads collapses into one query q_bar = sm_scale/H * sum_h q~_h, computed once
+// per request, and scoring streams the compressed cache once with one fp32 dot per entry.
+//
+// Kernels, in stream order:
+//   qbar_kernel     per request: q_bar, candidate count, reset of the selection state
+//   score_kernel    persistent, HBM-bound: streams every candidate entry with 16-byte
+//                   non-allocating loads, writes its fp32 score, and counts the top 11 bits of
+//                   its order key into a per-request histogram (first radix digit)
+//   topk_mark       per (request, 8192 scores): marks scores above the boundary bin in a
+//                   bitmap and appends boundary-bin candidates to a list
+//   topk_finish     per request: resolves the boundary bin with two more radix digits (and the
+//                   lower-index tie rule), then compacts the bitmap into ascending indices.
+
+#include "ckv_internal.h"
+
+namespace ckv {
+
+int64_t score_stride(int ratio, int max_seq_len) {
+  const int64_t n = static_cast<int64_t>(max_seq_len) / ratio;
+  return (n + 63) / 64 * 64;
+}
+
+IndexerWs indexer_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len) {
+  IndexerWs w{};
+  const int64_t stride = score_stride(p.r, max_seq_len);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return static_cast<char*>(base) + o;
+  };
+  const bool have = base != nullptr;
+  char* q = take(sizeof(float) * batch * p.D);
+  char* nc = take(sizeof(int32_t) * batch);
+  char* h = take(sizeof(uint32_t) * batch * kHistBins);
+  char* cc = take(sizeof(uint32_t) * batch);
+  char* bm = take(sizeof(uint32_t) * batch * (stride / 32));
+  char* cd = take(sizeof(uint2) * batch * stride);
+  char* sc = take(sizeof(float) * batch * stride);
+  if (have) {
+    w.qbar = reinterpret_cast<float*>(q);
+    w.n_c = reinterpret_cast<int32_t*>(nc);
+    w.hist = reinterpret_cast<uint32_t*>(h);
+    w.cand_cnt = reinterpret_cast<uint32_t*>(cc);
+    w.bitmap = reinterpret_cast<uint32_t*>(bm);
+    w.cand = reinterpret_cast<uint2*>(cd);
+    w.scores = reinterpret_cast<float*>(sc);
+  }
+  w.bytes = off;
+  return w;
+}
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMarkChunk = 8192;
+constexpr int kFinishThreads = 1024;
+
+// ---------------------------------------------------------------------------- block scans
+
+// inclusive scan of one value per thread across the block (blockDim.x multiple of 32)
+template <typename T>
+__device__ T block_inclusive_scan(T v, T* sh /* >= 32 */, T* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const T t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  __syncthreads();
+  if (lane == 31) sh[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    T s = lane < nw ? sh[lane] : T(0);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const T t = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += t;
+    }
+    if (lane < nw) sh[lane] = s;
+  }
+  __syncthreads();
+  if (w > 0) v += sh[w - 1];
+  if (total) *total = sh[nw - 1];
+  __syncthreads();
+  return v;
+}
+
+// Boundary of a histogram h[nbins] (shared or global) for selecting `need` items, scanning from
+// the top bin down (descending) or from bin 0 up: the bin where the running count reaches need,
+// and the count strictly before it in scan order. Result in out[0] (bin), out[1] (before).
+__device__ void find_boundary(const uint32_t* h, int nbins, uint32_t need, bool descending,
+                              uint32_t* sh /* >= 32 */, uint32_t* out) {
+  const int per = (nbins + blockDim.x - 1) / blockDim.x;
+  const int g0 = threadIdx.x * per;
+  uint32_t s = 0;
+  for (int i = 0; i < per; ++i) {
+    const int k = g0 + i;
+    if (k < nbins) s += h[descending ? nbins - 1 - k : k];
+  }
+  const uint32_t incl = block_inclusive_scan<uint32_t>(s, sh, nullptr);
+  const uint32_t excl = incl - s;
+  if (excl < need && incl >= need) {
+    uint32_t cum = excl;
+    for (int i = 0; i < per; ++i) {
+      const int k = g0 + i;
+      if (k >= nbins) break;
+      const int bin = descending ? nbins - 1 - k : k;
+      if (cum + h[bin] >= need) {
+        out[0] = bin;
+        out[1] = cum;
+        break;
+      }
+      cum += h[bin];
+    }
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------- q_bar
+
+__global__ void __launch_bounds__(kThreads) qbar_kernel(LayerParams p, const int32_t* seq_len,
+                                                        int max_seq_len, const float* q,
+                                                        IndexerWs ws, uint32_t* status) {
+  const int b = blockIdx.x;
+  const int L = seq_len[b];
+  const bool ok = L >= 1 && L <= max_seq_len;
+  if (threadIdx.x == 0) {
+    if (!ok) atomicOr(status, CKV_DEV_BAD_LENGTH);
+    ws.n_c[b] = ok ? L / p.r : 0;
+    ws.cand_cnt[b] = 0;
+  }
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ws.hist[static_cast<int64_t>(b) * kHistBins + i] = 0;
+  const int npairs = p.D / 2, first_rope = (p.D - p.d_r) / 2;
+  const float* qb = q + static_cast<int64_t>(b) * p.H * p.D;
+  const double scale = static_cast<double>(p.sm_scale) / p.H;
+  for (int pr = threadIdx.x; pr < npairs; pr += blockDim.x) {
+    double s0 = 0.0, s1 = 0.0;
+    for (int h = 0; h < p.H; ++h) {
+      const float2 v = reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h) * p.D)[pr];
+      s0 += v.x;
+      s1 += v.y;
+    }
+    if (pr >= first_rope && ok)
+      rope_rotate_pair(s0, s1, static_cast<double>(L - 1),
+                       rope_inv_freq(pr - first_rope, p.d_r, p.rope_base), false, &s0, &s1);
+    reinterpret_cast<float2*>(ws.qbar + static_cast<int64_t>(b) * p.D)[pr] =
+        make_float2(static_cast<float>(s0 * scale), static_cast<float>(s1 * scale));
+  }
+}
+
+// ---------------------------------------------------------------------------- scoring
+
+template <int DT>
+struct VecFmt;  // elements decoded from one 16-byte vector of codes
+template <> struct VecFmt<CKV_F32> { static constexpr int kElems = 4; };
+template <> struct VecFmt<CKV_BF16> { static constexpr int kElems = 8; };
+template <> struct VecFmt<CKV_NVFP4> { static constexpr int kElems = 32; };
+
+// dot of one 16-byte code vector with the matching q_bar elements held in registers
+template <int DT>
+__device__ __forceinline__ float vec_dot(const float* qv, uint4 raw, uint32_t sc16) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  float acc = 0.f;
+  if constexpr (DT == CKV_F32) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc = fmaf(qv[i], __uint_as_float(w[i]), acc);
+  } else if constexpr (DT == CKV_BF16) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc = fmaf(qv[2 * i], __uint_as_float(w[i] << 16), acc);
+      acc = fmaf(qv[2 * i + 1], __uint_as_float(w[i] & 0xffff0000u), acc);
+    }
+  } else {  // NVFP4: two 16-element blocks, each with its e4m3 scale
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk) {
+      float part = 0.f;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t word = w[2 * blk + i];
+#pragma unroll
+        for (int by = 0; by < 4; ++by) {
+          const float2 v = __half22float2(e2m1x2_to_half2(static_cast<uint8_t>(word >> (8 * by))));
+          const int e = 16 * blk + 8 * i + 2 * by;
+          part = fmaf(qv[e], v.x, part);
+          part = fmaf(qv[e + 1], v.y, part);
+        }
+      }
+      acc = fmaf(part, e4m3_to_f32(static_cast<uint8_t>(sc16 >> (8 * blk))), acc);
+    }
+  }
+  return acc;
+}
+
+// NV: 16-byte code vectors per entry (a power of two); U: entries per lane group per chunk
+template <int DT, int NV, int U>
+__global__ void __launch_bounds__(kThreads) score_kernel(LayerParams p, int batch, IndexerWs ws,
+                                                         float* scores, int64_t stride,
+                                                         uint32_t* status) {
+  constexpr int LPE = NV < 32 ? NV : 32;  // lanes per entry
+  constexpr int VPL = NV / LPE;           // vectors per lane per entry
+  constexpr int EPP = 32 / LPE;           // entries per warp pass
+  constexpr int CH = U * EPP;             // entries per warp chunk
+  constexpr int EPV = VecFmt<DT>::kElems;
+  static_assert(U <= LPE, "one writer lane per entry of a pass");
+
+  extern __shared__ int32_t chunk_prefix[];  // [batch + 1]
+  __shared__ int32_t scan_sh[32];
+  // chunks per request, exclusive prefix over the batch
+  {
+    const int per = (batch + blockDim.x - 1) / blockDim.x;
+    int32_t s = 0;
+    for (int i = 0; i < per; ++i) {
+      const int bb = threadIdx.x * per + i;
+      if (bb < batch) s += (ws.n_c[bb] + CH - 1) / CH;
+    }
+    int32_t total;
+    const int32_t incl = block_inclusive_scan<int32_t>(s, scan_sh, &total);
+    int32_t run = incl - s;
+    for (int i = 0; i < per; ++i) {
+      const int bb = threadIdx.x * per + i;
+      if (bb < batch) {
+        chunk_prefix[bb] = run;
+        run += (ws.n_c[bb] + CH - 1) / CH;
+      }
+    }
+    if (threadIdx.x == 0) chunk_prefix[batch] = total;
+    __syncthreads();
+  }
+  const int64_t total = chunk_prefix[batch];
+  const int64_t c_lo = total * blockIdx.x / gridDim.x;
+  const int64_t c_hi = total * (blockIdx.x + 1) / gridDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane % LPE, slot = lane / LPE;
+  const int sc_bytes = p.D / 16;
+
+  int cur_b = -1;
+  float qreg[VPL][EPV];
+  for (int64_t ch = c_lo + warp; ch < c_hi; ch += kWarps) {
+    // request of this chunk: last b with chunk_prefix[b] <= ch
+    int lo = 0, hi = batch;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (chunk_prefix[mid] <= ch) lo = mid; else hi = mid;
+    }
+    const int b = lo;
+    if (b != cur_b) {
+      const float* qb = ws.qbar + static_cast<int64_t>(b) * p.D;
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) {
+#pragma unroll
+        for (int e = 0; e < EPV; e += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(qb + (sub + LPE * k) * EPV + e);
+          qreg[k][e] = v.x; qreg[k][e + 1] = v.y; qreg[k][e + 2] = v.z; qreg[k][e + 3] = v.w;
+        }
+      }
+      cur_b = b;
+    }
+    const int N = ws.n_c[b];
+    const int64_t e_base = (ch - chunk_prefix[b]) * CH;
+    uint4 raw[U][VPL];
+    uint32_t sc[U][VPL];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t e = e_base + u * EPP + slot;
+      int64_t row = -1;
+      if (e < N) row = comp_row(p, b, e, status);
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) {
+        const int v = sub + LPE * k;
+        if (row >= 0) {
+          raw[u][k] = ldg_stream(p.comp_codes + row * p.comp_row_bytes + v * 16);
+          sc[u][k] = (DT == CKV_NVFP4)
+              ? static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p.comp_scales + row * sc_bytes + 2 * v))
+              : 0u;
+        } else {
+          raw[u][k] = make_uint4(0, 0, 0, 0);
+          sc[u][k] = 0u;
+        }
+      }
+    }
+    float acc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      acc[u] = 0.f;
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) acc[u] += vec_dot<DT>(qreg[k], raw[u][k], sc[u][k]);
+#pragma unroll
+      for (int o = LPE / 2; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+    }
+    // lane (slot, sub = u) writes the score of entry (pass u, slot) and counts its digit
+    float mine = 0.f;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (u == sub) mine = acc[u];
+    const int64_t e = e_base + static_cast<int64_t>(sub) * EPP + slot;
+    const bool writer = sub < U && e < N;
+    uint32_t bin = 0xffffffffu - lane;
+    if (writer) {
+      scores[static_cast<int64_t>(b) * stride + e] = mine;
+      bin = f32_order_key(mine) >> 21;
+    }
+    const uint32_t same = __match_any_sync(0xffffffffu, bin);
+    if (writer && lane == __ffs(same) - 1)
+      atomicAdd(ws.hist + static_cast<int64_t>(b) * kHistBins + bin, static_cast<uint32_t>(__popc(same)));
+  }
+}
+
+// ---------------------------------------------------------------------------- selection
+
+__global__ void __launch_bounds__(kThreads) topk_mark_kernel(const float* scores, int64_t stride,
+                                                             int top_k, IndexerWs ws) {
+  const int b = blockIdx.y;
+  const int64_t N = ws.n_c[b];
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * kMarkChunk;
+  if (j0 >= N) return;
+  const int64_t j1 = min(N, j0 + kMarkChunk);
+  uint32_t* bm = ws.bitmap + static_cast<int64_t>(b) * (stride / 32);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (N <= top_k) {  // every candidate is selected
+    for (int64_t w = j0 / 32 + threadIdx.x; w * 32 < j1; w += blockDim.x) {
+      const int64_t n = min(static_cast<int64_t>(32), N - w * 32);
+      bm[w] = n == 32 ? 0xffffffffu : ((1u << n) - 1u);
+    }
+    return;
+  }
+  __shared__ uint32_t sh[32];
+  __shared__ uint32_t bnd[2];
+  find_boundary(ws.hist + static_cast<int64_t>(b) * kHistBins, kHistBins, static_cast<uint32_t>(top_k),
+                true, sh, bnd);
+  const uint32_t b1 = bnd[0];
+  const float* sb = scores + static_cast<int64_t>(b) * stride;
+  uint2* cand = ws.cand + static_cast<int64_t>(b) * stride;
+  for (int64_t w = j0 / 32 + warp; w * 32 < j1; w += kWarps) {
+    const int64_t j = w * 32 + lane;
+    const bool in = j < j1;
+    const uint32_t key = in ? f32_order_key(sb[j]) : 0u;
+    const uint32_t bin = key >> 21;
+    const bool sel = in && bin > b1;
+    const bool cnd = in && bin == b1;
+    const uint32_t word = __ballot_sync(0xffffffffu, sel);
+    if (lane == 0) bm[w] = word;
+    const uint32_t cm = __ballot_sync(0xffffffffu, cnd);
+    if (cm) {
+      uint32_t base = 0;
+      if (lane == 0) base = atomicAdd(ws.cand_cnt + b, static_cast<uint32_t>(__popc(cm)));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (cnd) cand[base + __popc(cm & ((1u << lane) - 1u))] = make_uint2(key, static_cast<uint32_t>(j));
+    }
+  }
+}
+
+// Radix digit pass over the candidate list: histogram of digit(key) among items matching
+// `prefix` on the bits above `shift + width`, then the boundary for `need` from the top.
+struct DigitSel {
+  uint32_t bin, before;
+};
+
+template <bool kByIndex>
+__device__ DigitSel candidate_digit_pass(const uint2* cand, uint32_t m, uint32_t* h, int shift,
+                                         int width, uint32_t match_mask, uint32_t match_val,
+                                         uint32_t eq_key, uint32_t need, uint32_t* sh) {
+  const int nbins = 1 << width;
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < m; i += blockDim.x) {
+    const uint2 c = cand[i];
+    // by key: digits of the key, descending; by index: among key == eq_key, digits of the
+    // index, ascending
+    if (kByIndex && c.x != eq_key) continue;
+    const uint32_t v = kByIndex ? c.y : c.x;
+    if ((v & match_mask) != match_val) continue;
+    atomicAdd(h + ((v >> shift) & (nbins - 1)), 1u);
+  }
+  __syncthreads();
+  __shared__ uint32_t out[2];
+  find_boundary(h, nbins, need, !kByIndex, sh, out);
+  return DigitSel{out[0], out[1]};
+}
+
+__global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, IndexerWs ws,
+                                                                     int64_t stride, int32_t* idx,
+                                                                     int32_t* cnt) {
+  __shared__ uint32_t h[kHistBins];
+  __shared__ uint32_t sh[32];
+  __shared__ uint32_t bnd[2];
+  const int b = blockIdx.x;
+  const int64_t N = ws.n_c[b];
+  const int64_t k_eff = min(static_cast<int64_t>(top_k), N);
+  uint32_t* bm = ws.bitmap + static_cast<int64_t>(b) * (stride / 32);
+  if (N > top_k) {
+    find_boundary(ws.hist + static_cast<int64_t>(b) * kHistBins, kHistBins, static_cast<uint32_t>(top_k),
+                  true, sh, bnd);
+    const uint32_t b1 = bnd[0];
+    uint32_t need = static_cast<uint32_t>(k_eff) - bnd[1];
+    const uint32_t m = ws.cand_cnt[b];
+    const uint2* cand = ws.cand + static_cast<int64_t>(b) * stride;
+    // digits 2 and 3 of the key: bits [20:10] and [9:0]
+    const DigitSel dA = candidate_digit_pass<false>(cand, m, h, 10, 11, 0xffe00000u, b1 << 21, 0, need, sh);
+    need -= dA.before;
+    const uint32_t pA = (b1 << 21) | (dA.bin << 10);
+    const DigitSel dB = candidate_digit_pass<false>(cand, m, h, 0, 10, 0xfffffc00u, pA, 0, need, sh);
+    need -= dB.before;
+    const uint32_t T = pA | dB.bin;
+    const uint32_t n_eq = h[dB.bin];
+    // among key == T keep the `need` lowest indices: index threshold by three ascending digits
+    uint32_t idx_thr = 0xffffffffu;
+    if (need < n_eq) {
+      const DigitSel i1 = candidate_digit_pass<true>(cand, m, h, 21, 11, 0u, 0u, T, need, sh);
+      uint32_t nd = need - i1.before;
+      const uint32_t q1 = i1.bin << 21;
+      const DigitSel i2 = candidate_digit_pass<true>(cand, m, h, 10, 11, 0xffe00000u, q1, T, nd, sh);
+      nd -= i2.before;
+      const uint32_t q2 = q1 | (i2.bin << 10);
+      const DigitSel i3 = candidate_digit_pass<true>(cand, m, h, 0, 10, 0xfffffc00u, q2, T, nd, sh);
+      idx_thr = q2 | i3.bin;
+    }
+    for (uint32_t i = threadIdx.x; i < m; i += blockDim.x) {
+      const uint2 c = cand[i];
+      if (c.x > T || (c.x == T && c.y <= idx_thr)) atomicOr(bm + (c.y >> 5), 1u << (c.y & 31));
+    }
+    __threadfence_block();
+    __syncthreads();
+  }
+  // compaction of the bitmap into ascending indices
+  const int64_t nw = (N + 31) / 32;
+  const int64_t w0 = nw * threadIdx.x / blockDim.x, w1 = nw * (threadIdx.x + 1) / blockDim.x;
+  uint32_t c = 0;
+  for (int64_t w = w0; w < w1; ++w) c += __popc(__ldcg(bm + w));
+  const uint32_t incl = block_inclusive_scan<uint32_t>(c, sh, nullptr);
+  int64_t pos = incl - c;
+  int32_t* out = idx + static_cast<int64_t>(b) * top_k;
+  for (int64_t w = w0; w < w1; ++w) {
+    uint32_t word = __ldcg(bm + w);
+    while (word) {
+      const int bit = __ffs(word) - 1;
+      word &= word - 1;
+      if (pos < top_k) out[pos] = static_cast<int32_t>(w * 32 + bit);
+      ++pos;
+    }
+  }
+  for (int64_t i = k_eff + threadIdx.x; i < top_k; i += blockDim.x) out[i] = -1;
+  if (threadIdx.x == 0) cnt[b] = static_cast<int32_t>(k_eff);
+}
+
+template <int DT, int NV, int U>
+cudaError_t launch_score(const LayerParams& p, int batch, int max_seq_len, const IndexerWs& ws,
+                         float* scores, int64_t stride, uint32_t* status, cudaStream_t stream) {
+  constexpr int LPE = NV < 32 ? NV : 32;
+  constexpr int CH = U * (32 / LPE);
+  const int64_t per_req = (static_cast<int64_t>(max_seq_len) / p.r + CH - 1) / CH;
+  const int64_t chunks = per_req * batch;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 4 * kWarps;  // warps resident
+  int64_t grid = (chunks + kWarps - 1) / kWarps;
+  if (grid > cap / kWarps) grid = cap / kWarps;
+  if (grid < 1) grid = 1;
+  const int smem = static_cast<int>(sizeof(int32_t) * (batch + 1));
+  auto kern = score_kernel<DT, NV, U>;
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  prof_begin(kProfScore, stream);
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(p, batch, ws, scores, stride, status);
+  prof_end(kProfScore, stream);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int DT>
+cudaError_t dispatch_score(const LayerParams& p, int batch, int max_seq_len, const IndexerWs& ws,
+                           float* scores, int64_t stride, uint32_t* status, cudaStream_t stream) {
+  // 16-byte vectors per entry for D = 64 .. 1024: f32 D/4, bf16 D/8, nvfp4 D/32
+  const int nv = p.comp_row_bytes / 16;
+  constexpr int kMin = DT == CKV_F32 ? 16 : DT == CKV_BF16 ? 8 : 2;
+#define CKV_SCORE_CASE(M)                                                                    \
+  case kMin * M:                                                                             \
+    return launch_score<DT, kMin * M, (kMin * M < 8 ? kMin * M : 8)>(p, batch, max_seq_len,  \
+                                                                    ws, scores, stride,      \
+                                                                    status, stream);
+  switch (nv) {
+    CKV_SCORE_CASE(1)
+    CKV_SCORE_CASE(2)
+    CKV_SCORE_CASE(4)
+    CKV_SCORE_CASE(8)
+    CKV_SCORE_CASE(16)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef CKV_SCORE_CASE
+}
+
+}  // namespace
+
+cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
+                           int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
+                           float* scores, const IndexerWs& ws, uint32_t* status,
+                           cudaStream_t stream) {
+  const int64_t stride = score_stride(p.r, max_seq_len);
+  float* sc = scores ? scores : ws.scores;
+  qbar_kernel<<<batch, kThreads, 0, stream>>>(p, seq_len, max_seq_len, q, ws, status);
+  note_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  switch (p.comp_dtype) {
+    case CKV_F32: e = dispatch_score<CKV_F32>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
+    case CKV_BF16: e = dispatch_score<CKV_BF16>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
+    case CKV_NVFP4: e = dispatch_score<CKV_NVFP4>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
+    default: e = cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  const int64_t nmax = static_cast<int64_t>(max_seq_len) / p.r;
+  dim3 mgrid(static_cast<unsigned>(nmax > 0 ? (nmax + kMarkChunk - 1) / kMarkChunk : 1), batch);
+  topk_mark_kernel<<<mgrid, kThreads, 0, stream>>>(sc, stride, top_k, ws);
+  note_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  topk_finish_kernel<<<batch, kFinishThreads, 0, stream>>>(top_k, ws, stride, idx, cnt);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace ckv

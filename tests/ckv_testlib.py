@@ -6,6 +6,7 @@ Nothing here computes the method: the oracle and the CUDA binding each do their 
 from __future__ import annotations
 
 import numpy as np
+import torch
 
 from oracle import ckv_oracle as O
 from synth import workloads as S
@@ -83,3 +84,37 @@ def max_rel_err(out, ref):
     num = np.max(np.abs(out - ref), axis=-1)
     den = np.maximum(np.max(np.abs(ref), axis=-1), 1e-30)
     return float(np.max(num / den))
+
+
+# ------------------------------------------------------------------------------------------------
+# CUDA side (through the Python binding of the C ABI)
+# ------------------------------------------------------------------------------------------------
+
+def gpu_layer(ckv, w: S.Workload, lay: dict, ls: S.LayerSpec, max_seq_len=None, top_k="spec"):
+    """A DecodeLayer over copies of the generated pools (the tables are shared)."""
+    cfg = ckv.LayerConfig(w.num_heads, w.head_dim, w.rope_dim, ls.ratio, w.window, ls.comp_dtype,
+                          ls.win_dtype)
+    clone = lambda t: None if t is None else t.clone()  # noqa: E731
+    cache = ckv.cache_from_tensors(cfg, w.batch, clone(lay["comp_codes"]), clone(lay["comp_scales"]),
+                                   clone(lay["win_codes"]), clone(lay["win_scales"]),
+                                   lay["comp_table"], lay["win_table"])
+    msl = max(w.seq_lens) if max_seq_len is None else max_seq_len
+    return ckv.DecodeLayer(cfg, cache, w.batch, msl, ls.top_k if top_k == "spec" else top_k)
+
+
+def gpu_setup(dl, lay: dict) -> None:
+    cu = lay["cu_setup"]
+    n = (cu[1:] - cu[:-1]).max().item()
+    if n > 0:
+        dl.append(lay["setup_start"].to(torch.int32), lay["kv_setup"], lay["logit_setup"],
+                  cu_new=cu, max_new=int(n))
+
+
+def gpu_append_decode_token(dl, lay: dict, seq_len) -> None:
+    dl.append((seq_len - 1).to(torch.int32), lay["kv_new"], lay["logit_new"])
+
+
+def status_word(dl) -> int:
+    torch.cuda.synchronize()
+    return int(dl.status[0].item()) & 0xffffffff
+
