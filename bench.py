@@ -237,6 +237,10 @@ def run_cuda(args, w: S.Workload):
           for _ in range(args.steps)]
     kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(n_dom)] for _ in range(args.steps)]
+    for pair in ev + [x for row in kev for x in row]:   # torch creates CUDA events on first record
+        for e in pair:
+            e.record(stream)
+    torch.cuda.synchronize()
     clocks = ClockSampler(local)
     time.sleep(0.3)
     launches0 = ckv.launch_count()
@@ -417,7 +421,7 @@ def cpu_baseline(w, step, seconds):
             oracle_request(w, gen_host, li, b, O)
             reqs.append((li, b))
         done += 1
-        if time.perf_counter() - t0 >= seconds or done >= 4 * w.batch:
+        if time.perf_counter() - t0 >= seconds or done >= 64 * w.batch:
             break
     el = time.perf_counter() - t0
     return {"value": done * len(w.layers) / el, "unit": UNIT, "cores": oracle_threads(),
@@ -464,8 +468,8 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(S.WORKLOADS))
     ap.add_argument("--impl", default="ckv", choices=["ckv", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

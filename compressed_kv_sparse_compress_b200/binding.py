@@ -26,6 +26,7 @@ CKV_ERR_CUDA = -5
 CKV_DEV_BAD_BLOCK = 0x1
 CKV_DEV_BAD_LENGTH = 0x2
 CKV_DEV_BAD_INDEX = 0x4
+CKV_DEV_TIMEOUT = 0x8
 
 CKV_F32, CKV_BF16, CKV_FP8_E4M3, CKV_NVFP4 = 0, 1, 2, 3
 DTYPES = {"f32": CKV_F32, "bf16": CKV_BF16, "fp8": CKV_FP8_E4M3, "nvfp4": CKV_NVFP4}

@@ -190,6 +190,8 @@ __device__ void process_group(const AppendArgs& a, int b, int64_t g, int64_t pre
 }
 
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
+  griddep_wait();
+  griddep_launch();
   __shared__ float smem[256 + 1024 + 32];
   const int b = blockIdx.y;
   const int64_t prev = a.prev_len[b];
@@ -231,9 +233,7 @@ cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_l
   const int64_t groups = static_cast<int64_t>(max_new) / p.r + 2;
   const int gx = static_cast<int>(groups < 512 ? groups : 512);
   dim3 grid(gx, batch);
-  append_kernel<<<grid, kAppendThreads, 0, stream>>>(a);
-  note_launch();
-  return cudaGetLastError();
+  return launch_kernel(append_kernel, grid, dim3(kAppendThreads), 0, stream, a);
 }
 
 }  // namespace ckv

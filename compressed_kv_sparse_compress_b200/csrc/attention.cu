@@ -19,7 +19,8 @@
 namespace ckv {
 
 bool attention_tc_supported(const LayerParams& p);
-int attention_tc_keys_per_split();
+int attention_tc_tiles_per_split(int batch, int64_t max_keys);
+int attention_tc_tile_keys();
 cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,
                                 int max_seq_len, const float* q, const int32_t* idx,
                                 const int32_t* cnt, int idx_stride, const AttnWs& ws,
@@ -70,6 +71,8 @@ template <int D>
 __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const float* q, const int32_t* idx,
     const int32_t* cnt, int idx_stride, AttnWs ws, uint32_t* status) {
+  griddep_wait();
+  griddep_launch();
   constexpr int NPL = D / 64;  // rotary-aligned pairs per lane
   extern __shared__ float xs[];  // [kSimtKeys][D]
   __shared__ int valid[kSimtKeys];
@@ -158,6 +161,8 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
 __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const int32_t* cnt, bool sparse,
     int idx_stride, AttnWs ws, float* out, uint32_t* status) {
+  griddep_wait();
+  griddep_launch();
   const int h = blockIdx.x, b = blockIdx.y;
   const int D = p.D;
   float* o = out + (static_cast<int64_t>(b) * p.H + h) * D;
@@ -214,9 +219,8 @@ cudaError_t launch_simt_d(const LayerParams& p, int batch, const int32_t* seq_le
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   dim3 grid(ws.splits, batch);
-  kern<<<grid, kSimtThreads, smem, stream>>>(p, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status);
-  note_launch();
-  return cudaGetLastError();
+  return launch_kernel(kern, grid, dim3(kSimtThreads), smem, stream, p, seq_len, max_seq_len, q, idx,
+                       cnt, idx_stride, ws, status);
 }
 
 }  // namespace
@@ -226,7 +230,9 @@ AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_
   AttnWs w{};
   const int64_t sel = max_selected > 0 ? max_selected : static_cast<int64_t>(max_seq_len) / p.r;
   const int64_t keys = sel + (p.W < max_seq_len ? p.W : max_seq_len);
-  w.keys_per_split = attention_tc_supported(p) ? attention_tc_keys_per_split() : kSimtKeys;
+  w.keys_per_split = attention_tc_supported(p)
+                         ? attention_tc_tile_keys() * attention_tc_tiles_per_split(batch, keys)
+                         : kSimtKeys;
   w.splits = static_cast<int>(keys > 0 ? (keys + w.keys_per_split - 1) / w.keys_per_split : 1);
   const size_t n_slot = static_cast<size_t>(batch) * w.splits * p.H;
   const size_t o_bytes = align_up(n_slot * p.D * sizeof(float), 256);
@@ -260,10 +266,8 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
   prof_end(kProfAttention, stream);
   if (e != cudaSuccess) return e;
   dim3 grid(p.H, batch);
-  attn_combine_kernel<<<grid, kCombineThreads, 0, stream>>>(p, seq_len, max_seq_len, cnt, idx != nullptr,
-                                                           idx_stride, ws, out, status);
-  note_launch();
-  return cudaGetLastError();
+  return launch_kernel(attn_combine_kernel, grid, dim3(kCombineThreads), 0, stream, p, seq_len,
+                       max_seq_len, cnt, idx != nullptr, idx_stride, ws, out, status);
 }
 
 }  // namespace ckv

@@ -127,6 +127,13 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Programmatic dependent launch: every kernel of the library starts with
+//   griddep_wait();      // the previous kernel in the stream has completed, its writes visible
+//   griddep_launch();    // the next kernel may be scheduled now (it waits the same way)
+// so a launch overlaps the previous kernel's tail while all memory accesses stay ordered.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 v;
   asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"

@@ -61,7 +61,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMarkChunk = 8192;
+constexpr int kMarkChunk = 4 * kThreads;  // scores per mark CTA
 constexpr int kFinishThreads = 1024;
 
 // ---------------------------------------------------------------------------- block scans
@@ -127,9 +127,16 @@ __device__ void find_boundary(const uint32_t* h, int nbins, uint32_t need, bool 
 
 // ---------------------------------------------------------------------------- q_bar
 
-__global__ void __launch_bounds__(kThreads) qbar_kernel(LayerParams p, const int32_t* seq_len,
-                                                        int max_seq_len, const float* q,
-                                                        IndexerWs ws, uint32_t* status) {
+// One CTA of 1024 threads per request: thread (pair, quarter) sums a quarter of the heads of one
+// rotary-aligned pair of dims in fp64; the quarters are added in shared memory.
+constexpr int kQbarThreads = 1024;
+
+__global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const int32_t* seq_len,
+                                                            int max_seq_len, const float* q,
+                                                            IndexerWs ws, uint32_t* status) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ double part[4][2][256];
   const int b = blockIdx.x;
   const int L = seq_len[b];
   const bool ok = L >= 1 && L <= max_seq_len;
@@ -142,18 +149,32 @@ __global__ void __launch_bounds__(kThreads) qbar_kernel(LayerParams p, const int
   const int npairs = p.D / 2, first_rope = (p.D - p.d_r) / 2;
   const float* qb = q + static_cast<int64_t>(b) * p.H * p.D;
   const double scale = static_cast<double>(p.sm_scale) / p.H;
-  for (int pr = threadIdx.x; pr < npairs; pr += blockDim.x) {
+  for (int pr0 = 0; pr0 < npairs; pr0 += 256) {   // D <= 1024: at most two rounds
+    const int pr = pr0 + (threadIdx.x & 255), qtr = threadIdx.x >> 8;
     double s0 = 0.0, s1 = 0.0;
-    for (int h = 0; h < p.H; ++h) {
-      const float2 v = reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h) * p.D)[pr];
-      s0 += v.x;
-      s1 += v.y;
+    if (pr < npairs) {
+      const int h_lo = (p.H * qtr) / 4, h_hi = (p.H * (qtr + 1)) / 4;
+#pragma unroll 16
+      for (int h = h_lo; h < h_hi; ++h) {
+        const float2 v = __ldg(reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h) * p.D) + pr);
+        s0 += v.x;
+        s1 += v.y;
+      }
     }
-    if (pr >= first_rope && ok)
-      rope_rotate_pair(s0, s1, static_cast<double>(L - 1),
-                       rope_inv_freq(pr - first_rope, p.d_r, p.rope_base), false, &s0, &s1);
-    reinterpret_cast<float2*>(ws.qbar + static_cast<int64_t>(b) * p.D)[pr] =
-        make_float2(static_cast<float>(s0 * scale), static_cast<float>(s1 * scale));
+    part[qtr][0][threadIdx.x & 255] = s0;
+    part[qtr][1][threadIdx.x & 255] = s1;
+    __syncthreads();
+    if (qtr == 0 && pr < npairs) {
+      const int k = threadIdx.x & 255;
+      s0 = (part[0][0][k] + part[1][0][k]) + (part[2][0][k] + part[3][0][k]);
+      s1 = (part[0][1][k] + part[1][1][k]) + (part[2][1][k] + part[3][1][k]);
+      if (pr >= first_rope && ok)
+        rope_rotate_pair(s0, s1, static_cast<double>(L - 1),
+                         rope_inv_freq(pr - first_rope, p.d_r, p.rope_base), false, &s0, &s1);
+      reinterpret_cast<float2*>(ws.qbar + static_cast<int64_t>(b) * p.D)[pr] =
+          make_float2(static_cast<float>(s0 * scale), static_cast<float>(s1 * scale));
+    }
+    __syncthreads();
   }
 }
 
@@ -205,6 +226,8 @@ template <int DT, int NV, int U>
 __global__ void __launch_bounds__(kThreads) score_kernel(LayerParams p, int batch, IndexerWs ws,
                                                          float* scores, int64_t stride,
                                                          uint32_t* status) {
+  griddep_wait();
+  griddep_launch();
   constexpr int LPE = NV < 32 ? NV : 32;  // lanes per entry
   constexpr int VPL = NV / LPE;           // vectors per lane per entry
   constexpr int EPP = 32 / LPE;           // entries per warp pass
@@ -316,45 +339,73 @@ __global__ void __launch_bounds__(kThreads) score_kernel(LayerParams p, int batc
 
 // ---------------------------------------------------------------------------- selection
 
+// One CTA per 1024 scores of a request: each lane classifies 4 consecutive scores against the
+// boundary bin of the first digit; the bitmap word of 32 scores is assembled from 8 lanes.
 __global__ void __launch_bounds__(kThreads) topk_mark_kernel(const float* scores, int64_t stride,
                                                              int top_k, IndexerWs ws) {
+  griddep_wait();
+  griddep_launch();
   const int b = blockIdx.y;
   const int64_t N = ws.n_c[b];
   const int64_t j0 = static_cast<int64_t>(blockIdx.x) * kMarkChunk;
   if (j0 >= N) return;
-  const int64_t j1 = min(N, j0 + kMarkChunk);
   uint32_t* bm = ws.bitmap + static_cast<int64_t>(b) * (stride / 32);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t j = j0 + 4 * static_cast<int64_t>(threadIdx.x);  // this lane's 4 scores
+  const int64_t w0 = (j0 >> 5) + 4 * warp;                        // this warp's 4 words
   if (N <= top_k) {  // every candidate is selected
-    for (int64_t w = j0 / 32 + threadIdx.x; w * 32 < j1; w += blockDim.x) {
-      const int64_t n = min(static_cast<int64_t>(32), N - w * 32);
-      bm[w] = n == 32 ? 0xffffffffu : ((1u << n) - 1u);
+    if (threadIdx.x < kMarkChunk / 32) {
+      const int64_t w = (j0 >> 5) + threadIdx.x;
+      if (w * 32 < N) {
+        const int64_t n = min(static_cast<int64_t>(32), N - w * 32);
+        bm[w] = n == 32 ? 0xffffffffu : ((1u << n) - 1u);
+      }
     }
     return;
   }
+  // the lane's scores (stride is a multiple of 64 floats, so the float4 is in bounds)
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (j < N) v = __ldcg(reinterpret_cast<const float4*>(scores + static_cast<int64_t>(b) * stride + j));
   __shared__ uint32_t sh[32];
   __shared__ uint32_t bnd[2];
   find_boundary(ws.hist + static_cast<int64_t>(b) * kHistBins, kHistBins, static_cast<uint32_t>(top_k),
                 true, sh, bnd);
   const uint32_t b1 = bnd[0];
-  const float* sb = scores + static_cast<int64_t>(b) * stride;
-  uint2* cand = ws.cand + static_cast<int64_t>(b) * stride;
-  for (int64_t w = j0 / 32 + warp; w * 32 < j1; w += kWarps) {
-    const int64_t j = w * 32 + lane;
-    const bool in = j < j1;
-    const uint32_t key = in ? f32_order_key(sb[j]) : 0u;
-    const uint32_t bin = key >> 21;
-    const bool sel = in && bin > b1;
-    const bool cnd = in && bin == b1;
-    const uint32_t word = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) bm[w] = word;
-    const uint32_t cm = __ballot_sync(0xffffffffu, cnd);
-    if (cm) {
-      uint32_t base = 0;
-      if (lane == 0) base = atomicAdd(ws.cand_cnt + b, static_cast<uint32_t>(__popc(cm)));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      if (cnd) cand[base + __popc(cm & ((1u << lane) - 1u))] = make_uint2(key, static_cast<uint32_t>(j));
-    }
+  const float vals[4] = {v.x, v.y, v.z, v.w};
+  uint32_t keys[4];
+  uint32_t sel = 0, cnd = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    keys[e] = f32_order_key(vals[e]);
+    const bool in = j + e < N;
+    const uint32_t bin = keys[e] >> 21;
+    if (in && bin > b1) sel |= 1u << e;
+    if (in && bin == b1) cnd |= 1u << e;
+  }
+  // bitmap: lanes 8k..8k+7 hold the 32 bits of word k of the warp
+  uint32_t word = sel << (4 * (lane & 7));
+  word |= __shfl_xor_sync(0xffffffffu, word, 1);
+  word |= __shfl_xor_sync(0xffffffffu, word, 2);
+  word |= __shfl_xor_sync(0xffffffffu, word, 4);
+  if ((lane & 7) == 0 && (w0 + (lane >> 3)) * 32 < N) bm[w0 + (lane >> 3)] = word;
+  // boundary-bin candidates: one atomic per warp, then each lane writes its own
+  const int mine = __popc(cnd);
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (total) {
+    uint32_t base = 0;
+    if (lane == 31) base = atomicAdd(ws.cand_cnt + b, static_cast<uint32_t>(total));
+    base = __shfl_sync(0xffffffffu, base, 31);
+    uint2* cand = ws.cand + static_cast<int64_t>(b) * stride;
+    uint32_t pos = base + incl - mine;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (cnd & (1u << e)) cand[pos++] = make_uint2(keys[e], static_cast<uint32_t>(j + e));
   }
 }
 
@@ -389,7 +440,11 @@ __device__ DigitSel candidate_digit_pass(const uint2* cand, uint32_t m, uint32_t
 __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, IndexerWs ws,
                                                                      int64_t stride, int32_t* idx,
                                                                      int32_t* cnt) {
+  griddep_wait();
+  griddep_launch();
+  constexpr uint32_t kCandSmem = 2048;  // boundary-bin candidates kept in shared memory
   __shared__ uint32_t h[kHistBins];
+  __shared__ uint2 cand_s[kCandSmem];
   __shared__ uint32_t sh[32];
   __shared__ uint32_t bnd[2];
   const int b = blockIdx.x;
@@ -403,6 +458,11 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, 
     uint32_t need = static_cast<uint32_t>(k_eff) - bnd[1];
     const uint32_t m = ws.cand_cnt[b];
     const uint2* cand = ws.cand + static_cast<int64_t>(b) * stride;
+    if (m <= kCandSmem) {
+      for (uint32_t i = threadIdx.x; i < m; i += blockDim.x) cand_s[i] = __ldcg(cand + i);
+      __syncthreads();
+      cand = cand_s;
+    }
     // digits 2 and 3 of the key: bits [20:10] and [9:0]
     const DigitSel dA = candidate_digit_pass<false>(cand, m, h, 10, 11, 0xffe00000u, b1 << 21, 0, need, sh);
     need -= dA.before;
@@ -467,10 +527,10 @@ cudaError_t launch_score(const LayerParams& p, int batch, int max_seq_len, const
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   prof_begin(kProfScore, stream);
-  kern<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(p, batch, ws, scores, stride, status);
+  e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, p, batch, ws,
+                    scores, stride, status);
   prof_end(kProfScore, stream);
-  note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 template <int DT>
@@ -504,9 +564,8 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
                            cudaStream_t stream) {
   const int64_t stride = score_stride(p.r, max_seq_len);
   float* sc = scores ? scores : ws.scores;
-  qbar_kernel<<<batch, kThreads, 0, stream>>>(p, seq_len, max_seq_len, q, ws, status);
-  note_launch();
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(qbar_kernel, dim3(batch), dim3(kQbarThreads), 0, stream, p, seq_len,
+                                max_seq_len, q, ws, status);
   if (e != cudaSuccess) return e;
   switch (p.comp_dtype) {
     case CKV_F32: e = dispatch_score<CKV_F32>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
@@ -517,12 +576,11 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
   if (e != cudaSuccess) return e;
   const int64_t nmax = static_cast<int64_t>(max_seq_len) / p.r;
   dim3 mgrid(static_cast<unsigned>(nmax > 0 ? (nmax + kMarkChunk - 1) / kMarkChunk : 1), batch);
-  topk_mark_kernel<<<mgrid, kThreads, 0, stream>>>(sc, stride, top_k, ws);
-  note_launch();
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  topk_finish_kernel<<<batch, kFinishThreads, 0, stream>>>(top_k, ws, stride, idx, cnt);
-  note_launch();
-  return cudaGetLastError();
+  e = launch_kernel(topk_mark_kernel, mgrid, dim3(kThreads), 0, stream, static_cast<const float*>(sc),
+                    stride, top_k, ws);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(topk_finish_kernel, dim3(batch), dim3(kFinishThreads), 0, stream, top_k, ws, stride,
+                       idx, cnt);
 }
 
 }  // namespace ckv

@@ -55,6 +55,8 @@ typedef enum {
 #define CKV_DEV_BAD_BLOCK 0x1u   /* a needed table entry was < 0 or >= the pool's block count  */
 #define CKV_DEV_BAD_LENGTH 0x2u  /* a length < 0 (append) / < 1 (decode) or > max_seq_len     */
 #define CKV_DEV_BAD_INDEX 0x4u   /* a selected entry index outside [0, floor(L/r))            */
+#define CKV_DEV_TIMEOUT 0x8u     /* a bounded wait for the tensor cores gave up (the split's
+                                    partial is marked empty)                                  */
 
 typedef enum {
   CKV_F32 = 0,       /* fp32                                                         */
