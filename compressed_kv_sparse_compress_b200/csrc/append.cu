@@ -51,16 +51,16 @@ __device__ __forceinline__ float2 rotate_raw_pair(const AppendArgs& a, const flo
   if (pr < first_rope_pair) return make_float2(x0, x1);
   double o0, o1;
   rope_rotate_pair(x0, x1, static_cast<double>(pos),
-                   rope_inv_freq(pr - first_rope_pair, p.d_r, p.rope_base), false, &o0, &o1);
+                   rope_inv_freq(p, pr - first_rope_pair), false, &o0, &o1);
   return make_float2(static_cast<float>(o0), static_cast<float>(o1));
 }
 
-// Writes one rotated token (pairs held by this thread) into the window cache.
-__device__ void write_window_token(const AppendArgs& a, int b, int64_t pos,
+// Writes one rotated token (pairs held by this thread) into window pool row `row` (skipped when
+// negative; the reduction still runs so that every thread reaches the same barriers).
+__device__ void write_window_token(const AppendArgs& a, int64_t row,
                                    const float2 (&x)[kMaxPairsPerThread], float* red) {
   const LayerParams& p = a.p;
   const int npairs = p.D / 2;
-  const int64_t row = win_row(p, b, pos, a.status);  // uniform across the block
   if (p.win_dtype == CKV_F32) {
     if (row < 0) return;
     float2* dst = reinterpret_cast<float2*>(p.win_codes + row * p.win_row_bytes);
@@ -129,10 +129,24 @@ __device__ void process_group(const AppendArgs& a, int b, int64_t g, int64_t pre
   float* ring = p.res_kv + static_cast<int64_t>(b) * r * D;
   float* ring_logit = p.res_logit + static_cast<int64_t>(b) * r;
 
+  // loads that do not depend on the new tokens first: the entry's pool row and the logits
+  int64_t crow = -1;
+  if (complete) {
+    crow = comp_row(p, b, g, a.status);
+    if (threadIdx.x < 32)
+      for (int t = threadIdx.x; t < r; t += 32) {
+        const int64_t pos = t0 + t;
+        w[t] = pos < prev ? ring_logit[pos % r] : a.logit_new[row0 + (pos - prev)];
+      }
+  }
+
   // new tokens of the group: window and (unfinished group) residue ring
+  float2 xlast[kMaxPairsPerThread];
+  int64_t pos_last = -1;
   for (int64_t pos = max(t0, prev); pos < t_end; ++pos) {
     const bool to_window = p.W > 0 && pos >= new_len - p.W;
-    if (!to_window && complete) continue;
+    if (!to_window && complete && pos != t_end - 1) continue;
+    const int64_t wrow = to_window ? win_row(p, b, pos, a.status) : -1;
     const float* raw = a.kv_new + (row0 + (pos - prev)) * D;
     float2 x[kMaxPairsPerThread];
     for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) x[k] = rotate_raw_pair(a, raw, pr, pos);
@@ -141,20 +155,18 @@ __device__ void process_group(const AppendArgs& a, int b, int64_t g, int64_t pre
       for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) dst[pr] = x[k];
       if (threadIdx.x == 0) ring_logit[pos % r] = a.logit_new[row0 + (pos - prev)];
     }
-    if (to_window) write_window_token(a, b, pos, x, red);
+    if (to_window) write_window_token(a, wrow, x, red);
+#pragma unroll
+    for (int k = 0; k < kMaxPairsPerThread; ++k) xlast[k] = x[k];
+    pos_last = pos;
   }
   if (!complete) return;
 
-  // softmax of the group's logits (positions before prev come from the ring)
+  // softmax of the group's logits
   __syncthreads();
   if (threadIdx.x < 32) {
     float m = -INFINITY;
-    for (int t = threadIdx.x; t < r; t += 32) {
-      const int64_t pos = t0 + t;
-      const float lg = pos < prev ? ring_logit[pos % r] : a.logit_new[row0 + (pos - prev)];
-      w[t] = lg;
-      m = fmaxf(m, lg);
-    }
+    for (int t = threadIdx.x; t < r; t += 32) m = fmaxf(m, w[t]);
     m = warp_max(m);
     float s = 0.f;
     for (int t = threadIdx.x; t < r; t += 32) {
@@ -167,25 +179,31 @@ __device__ void process_group(const AppendArgs& a, int b, int64_t g, int64_t pre
   }
   __syncthreads();
   // entry = sum over the group's tokens, in token order, of w_t * rotated token t
-  for (int pr = threadIdx.x; pr < npairs; pr += blockDim.x) {
+  for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) {
     float2 acc = make_float2(0.f, 0.f);
-    for (int t = 0; t < r; ++t) {
-      const int64_t pos = t0 + t;
-      float2 x;
-      if (pos < prev) {
-        x = reinterpret_cast<const float2*>(ring + (pos % r) * D)[pr];
-      } else {
-        x = rotate_raw_pair(a, a.kv_new + (row0 + (pos - prev)) * D, pr, pos);
+    for (int tb = 0; tb < r; tb += 4) {   // four tokens' loads in flight
+      float2 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t pos = t0 + tb + u;
+        if (tb + u >= r) x[u] = make_float2(0.f, 0.f);
+        else if (pos < prev) x[u] = reinterpret_cast<const float2*>(ring + (pos % r) * D)[pr];
+        else if (pos == pos_last) x[u] = xlast[k];
+        else x[u] = rotate_raw_pair(a, a.kv_new + (row0 + (pos - prev)) * D, pr, pos);
       }
-      acc.x = fmaf(w[t], x.x, acc.x);
-      acc.y = fmaf(w[t], x.y, acc.y);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (tb + u < r) {
+          acc.x = fmaf(w[tb + u], x[u].x, acc.x);
+          acc.y = fmaf(w[tb + u], x[u].y, acc.y);
+        }
+      }
     }
     c[2 * pr] = acc.x;
     c[2 * pr + 1] = acc.y;
   }
   __syncthreads();
-  const int64_t row = comp_row(p, b, g, a.status);
-  if (row >= 0) store_entry(p, row, c);
+  if (crow >= 0) store_entry(p, crow, c);
   __syncthreads();
 }
 

@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
       float2 v = reinterpret_cast<const float2*>(qh)[pr];
       if (pr >= first_rope) {
         double a, c;
-        rope_rotate_pair(v.x, v.y, pos, rope_inv_freq(pr - first_rope, p.d_r, p.rope_base), false, &a, &c);
+        rope_rotate_pair(v.x, v.y, pos, rope_inv_freq(p, pr - first_rope), false, &a, &c);
         v = make_float2(static_cast<float>(a), static_cast<float>(c));
       }
       qv[k] = v;
@@ -158,6 +158,76 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   }
 }
 
+// Per request: cos/sin of every rotary pair at the query position L-1 (fp64 angles), for the
+// inverse rotation in the combine; on the tensor-core path also the rotated query rounded to
+// fp16, written as the 128-byte-swizzled image of the MMA operand so that each attention CTA
+// fetches it with one bulk copy.
+constexpr int kPrepThreads = 256;
+
+__global__ void __launch_bounds__(kPrepThreads) attn_prep_kernel(LayerParams p, const int32_t* seq_len,
+                                                                 int max_seq_len, const float* q,
+                                                                 AttnWs ws) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ double rope_s[2 * 512];
+  const int b = blockIdx.x;
+  const int L = seq_len[b];
+  if (L < 1 || L > max_seq_len) return;
+  const int n_pairs = p.d_r / 2;
+  double* rope_g = ws.rope + static_cast<int64_t>(b) * (n_pairs + 1) * 2;
+  for (int i = threadIdx.x; i < n_pairs; i += blockDim.x) {
+    double sn, cs;
+    sincos(static_cast<double>(L - 1) * rope_inv_freq(p, i), &sn, &cs);
+    rope_s[2 * i] = cs;
+    rope_s[2 * i + 1] = sn;
+    rope_g[2 * i] = cs;
+    rope_g[2 * i + 1] = sn;
+  }
+  if (!ws.qimage) return;
+  __syncthreads();
+  // tensor-core path (H = 64, D = 512): granule g (8 dims) of head h lands at chunk g/8, row h,
+  // 16-byte slot (g % 8) ^ (h % 8) of the operand image
+  constexpr int kD = 512, kGr = kD / 8, kChunk = 64 * 128;
+  const float* qb = q + static_cast<int64_t>(b) * 64 * kD;
+  uint8_t* img = ws.qimage + static_cast<int64_t>(b) * kQImageBytes;
+  const int first_rope = (kD - p.d_r) / 2;
+  for (int it0 = 0; it0 < 64 * kGr; it0 += 8 * kPrepThreads) {
+    float4 raw[8][2];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int it = it0 + u * kPrepThreads + threadIdx.x;
+      const float4* src = reinterpret_cast<const float4*>(qb + (it >> 6) * kD + 8 * (it & 63));
+      raw[u][0] = __ldg(src);
+      raw[u][1] = __ldg(src + 1);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int it = it0 + u * kPrepThreads + threadIdx.x;
+      const int h = it >> 6, g = it & 63;
+      float v[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                    raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int pr = 4 * g + k;
+        if (pr >= first_rope) {
+          const double cs = rope_s[2 * (pr - first_rope)], sn = rope_s[2 * (pr - first_rope) + 1];
+          const double x0 = v[2 * k], x1 = v[2 * k + 1];
+          v[2 * k] = static_cast<float>(x0 * cs - x1 * sn);
+          v[2 * k + 1] = static_cast<float>(x0 * sn + x1 * cs);
+        }
+      }
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __half2 hh = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+        w[k] = *reinterpret_cast<uint32_t*>(&hh);
+      }
+      const uint32_t off = static_cast<uint32_t>(g >> 3) * kChunk + h * 128 + (((g & 7) ^ (h & 7)) << 4);
+      *reinterpret_cast<uint4*>(img + off) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const int32_t* cnt, bool sparse,
     int idx_stride, AttnWs ws, float* out, uint32_t* status) {
@@ -174,37 +244,64 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(
   }
   const KeyList kl = key_list(p, L, cnt, sparse, idx_stride, b);
   const int ns = static_cast<int>((kl.n_keys + ws.keys_per_split - 1) / ws.keys_per_split);
+  // log-sum-exp merge of the splits: M = max of the split maxima, Z = sum l_s exp(m_s - M)
+  __shared__ float red_m[32], red_z[32];
   const float2* ml = reinterpret_cast<const float2*>(ws.part_ml);
   const int64_t base = static_cast<int64_t>(b) * ws.splits;
+  float mloc = -INFINITY;
+  for (int s = threadIdx.x; s < ns; s += blockDim.x) {
+    const float2 v = __ldcg(ml + (base + s) * p.H + h);
+    if (v.y > 0.f) mloc = fmaxf(mloc, v.x);
+  }
+  mloc = warp_max(mloc);
+  if ((threadIdx.x & 31) == 0) red_m[threadIdx.x >> 5] = mloc;
+  __syncthreads();
   float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) {
-    const float2 v = ml[(base + s) * p.H + h];
-    if (v.y > 0.f) M = fmaxf(M, v.x);
+  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) M = fmaxf(M, red_m[i]);
+  float zloc = 0.f;
+  for (int s = threadIdx.x; s < ns; s += blockDim.x) {
+    const float2 v = __ldcg(ml + (base + s) * p.H + h);
+    if (v.y > 0.f) zloc += v.y * expf(v.x - M);
   }
+  zloc = warp_sum(zloc);
+  if ((threadIdx.x & 31) == 0) red_z[threadIdx.x >> 5] = zloc;
+  __syncthreads();
   float Z = 0.f;
-  for (int s = 0; s < ns; ++s) {
-    const float2 v = ml[(base + s) * p.H + h];
-    if (v.y > 0.f) Z += v.y * expf(v.x - M);
-  }
+  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) Z += red_z[i];
   const float inv = Z > 0.f ? 1.f / Z : 0.f;
   const int first_rope = (D - p.d_r) / 2;
+  const double* rope = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
+  const float* po = ws.part_o + (base * p.H + h) * D;
+  const int64_t split_stride = static_cast<int64_t>(p.H) * D;
   for (int pr = threadIdx.x; pr < D / 2; pr += blockDim.x) {
     float2 acc = make_float2(0.f, 0.f);
-    for (int s = 0; s < ns; ++s) {
-      const float2 v = ml[(base + s) * p.H + h];
-      if (!(v.y > 0.f)) continue;
-      const float w = expf(v.x - M);
-      const float2 x = reinterpret_cast<const float2*>(ws.part_o + ((base + s) * p.H + h) * D)[pr];
-      acc.x = fmaf(w, x.x, acc.x);
-      acc.y = fmaf(w, x.y, acc.y);
+    for (int s0 = 0; s0 < ns; s0 += 8) {   // eight splits' loads in flight
+      float wgt[8];
+      float2 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        wgt[u] = 0.f;
+        if (s0 + u < ns) {
+          const float2 v = __ldcg(ml + (base + s0 + u) * p.H + h);
+          if (v.y > 0.f) wgt[u] = expf(v.x - M);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        x[u] = wgt[u] > 0.f ? __ldcg(reinterpret_cast<const float2*>(po + (s0 + u) * split_stride) + pr)
+                            : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc.x = fmaf(wgt[u], x[u].x, acc.x);
+        acc.y = fmaf(wgt[u], x[u].y, acc.y);
+      }
     }
     acc.x *= inv;
     acc.y *= inv;
-    if (pr >= first_rope) {
-      double a, c;
-      rope_rotate_pair(acc.x, acc.y, static_cast<double>(L - 1),
-                       rope_inv_freq(pr - first_rope, p.d_r, p.rope_base), true, &a, &c);
-      acc = make_float2(static_cast<float>(a), static_cast<float>(c));
+    if (pr >= first_rope) {   // inverse rotation by the query position
+      const double cs = rope[2 * (pr - first_rope)], sn = rope[2 * (pr - first_rope) + 1];
+      const double a = acc.x, c = acc.y;
+      acc = make_float2(static_cast<float>(a * cs + c * sn), static_cast<float>(c * cs - a * sn));
     }
     reinterpret_cast<float2*>(o)[pr] = acc;
   }
@@ -237,11 +334,16 @@ AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_
   const size_t n_slot = static_cast<size_t>(batch) * w.splits * p.H;
   const size_t o_bytes = align_up(n_slot * p.D * sizeof(float), 256);
   const size_t ml_bytes = align_up(n_slot * 2 * sizeof(float), 256);
+  const size_t rope_bytes = align_up(static_cast<size_t>(batch) * (p.d_r / 2 + 1) * 2 * sizeof(double), 256);
+  const size_t q_bytes = attention_tc_supported(p) ? static_cast<size_t>(batch) * kQImageBytes : 0;
   if (base) {
-    w.part_o = static_cast<float*>(base);
-    w.part_ml = reinterpret_cast<float*>(static_cast<char*>(base) + o_bytes);
+    char* c = static_cast<char*>(base);
+    w.part_o = reinterpret_cast<float*>(c);
+    w.part_ml = reinterpret_cast<float*>(c + o_bytes);
+    w.rope = reinterpret_cast<double*>(c + o_bytes + ml_bytes);
+    w.qimage = q_bytes ? reinterpret_cast<uint8_t*>(c + o_bytes + ml_bytes + rope_bytes) : nullptr;
   }
-  w.bytes = o_bytes + ml_bytes;
+  w.bytes = o_bytes + ml_bytes + rope_bytes + q_bytes;
   return w;
 }
 
@@ -249,7 +351,9 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
                              int max_seq_len, const float* q, const int32_t* idx,
                              const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
                              uint32_t* status, cudaStream_t stream) {
-  cudaError_t e;
+  cudaError_t e = launch_kernel(attn_prep_kernel, dim3(batch), dim3(kPrepThreads), 0, stream, p, seq_len,
+                                max_seq_len, q, ws);
+  if (e != cudaSuccess) return e;
   prof_begin(kProfAttention, stream);
   if (attention_tc_supported(p)) {
     e = launch_attention_tc(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);

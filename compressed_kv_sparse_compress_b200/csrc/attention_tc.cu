@@ -25,6 +25,7 @@
 // merges the splits and applies the inverse rotation.
 
 #include "ckv_internal.h"
+#include "ckv_ptx.cuh"
 
 namespace ckv {
 namespace {
@@ -43,7 +44,6 @@ constexpr uint32_t kSCol = 0;
 constexpr uint32_t kOCol = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescale = 8.0f;
-constexpr uint32_t kWaitLimit = 1u << 22;
 
 // shared memory carve-up (byte offsets from a 1024-aligned base)
 constexpr uint32_t kOffX = 0;
@@ -67,18 +67,10 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 // ------------------------------------------------------------------------------------ PTX
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
                : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -87,43 +79,6 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(phase)
-      : "memory");
-  return ok != 0;
-}
-
-// bounded wait on an mbarrier phase; false after kWaitLimit polls
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, phase)) return true;
-  return false;
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-// global -> shared bulk copy (16-byte aligned, size a multiple of 16) completing on `bar`
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -360,20 +315,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   const int64_t k_end = min(n_keys, k_begin + ws.keys_per_split);
   const int n_tiles = static_cast<int>((k_end - k_begin + kTile - 1) / kTile);
 
-  // ---- set-up: barriers, raw query -> shared memory (bulk copy into the free X region), tile 0
-  //      key metadata, running statistics, rotary table, tensor memory
+  // ---- set-up: barriers; the prepared query image (64 KB, written per request by the prep
+  //      kernel) is bulk-copied into the Q region while the keys of tile 0 are resolved and staged
   const uint32_t bar_q = sb + kOffBarQ;
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(bar_q, 1);
     fence_proxy_async();
     flags[0] = flags[1] = 0;
-    const float* qb = q + static_cast<int64_t>(b) * kH * kD;
-    constexpr uint32_t kQRaw = kH * kD * 4, kPiece = 16384;
-    mbar_expect_tx(bar_q, kQRaw);
+    const uint8_t* img = ws.qimage + static_cast<int64_t>(b) * kQBytes;
+    constexpr uint32_t kPiece = 16384;
+    mbar_expect_tx(bar_q, kQBytes);
 #pragma unroll 1
-    for (uint32_t off = 0; off < kQRaw; off += kPiece)
-      bulk_g2s(sb + kOffX + off, reinterpret_cast<const uint8_t*>(qb) + off, kPiece, bar_q);
+    for (uint32_t off = 0; off < kQBytes; off += kPiece) bulk_g2s(sb + kOffQ + off, img + off, kPiece, bar_q);
   }
   key_meta<WT>(p, b, L, idx, idx_stride, n_c, n_sel, n_win, k_begin, k_end, key_row, key_win, key_vs,
                key_ls, status);
@@ -381,47 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     m_run[tid] = -INFINITY;
     l_run[tid] = 0.f;
   }
-  double* rope_cs = reinterpret_cast<double*>(base + kOffP);  // [pairs][2] (P is free here)
-  const int first_rope = (kD - p.d_r) / 2;
-  for (int i = tid; i < p.d_r / 2; i += kThreads) {
-    double sn, cs;
-    sincos(static_cast<double>(L - 1) * rope_inv_freq(i, p.d_r, p.rope_base), &sn, &cs);
-    rope_cs[2 * i] = cs;
-    rope_cs[2 * i + 1] = sn;
-  }
   if (warp == 0) tmem_alloc(sb + kOffTmem, kTmemCols);
-  __syncthreads();
-  bool ok = __syncthreads_and(mbar_wait(bar_q, 0)) != 0;
-
-  // ---- Q~ = rotated query, fp16, K-major swizzled [64 heads][512]
-  if (ok) {
-    const float* qs = reinterpret_cast<const float*>(base + kOffX);
-#pragma unroll 4
-    for (int it = tid; it < kH * (kD / 8); it += kThreads) {
-      const int h = it >> 6, g = it & 63;
-      const float4 a = reinterpret_cast<const float4*>(qs + h * kD + 8 * g)[0];
-      const float4 c = reinterpret_cast<const float4*>(qs + h * kD + 8 * g)[1];
-      float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int pr = 4 * g + k;
-        if (pr >= first_rope) {
-          const double cs = rope_cs[2 * (pr - first_rope)], sn = rope_cs[2 * (pr - first_rope) + 1];
-          const double x0 = v[2 * k], x1 = v[2 * k + 1];
-          v[2 * k] = static_cast<float>(x0 * cs - x1 * sn);
-          v[2 * k + 1] = static_cast<float>(x0 * sn + x1 * cs);
-        }
-      }
-      st_shared_v4(sb + kOffQ + swz(kQChunk, h, g),
-                   make_uint4(pack_f32x2(v[0], v[1]), pack_f32x2(v[2], v[3]), pack_f32x2(v[4], v[5]),
-                              pack_f32x2(v[6], v[7])));
-    }
-  }
   tc_fence_before();
-  __syncthreads();   // the X region is free again once every thread has read the query
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   uint32_t phase = 0;
+  bool ok = true;
+  bool q_ready = false;
 
   for (int tile = 0; tile < n_tiles && ok; ++tile) {
     if (tile > 0) {
@@ -449,6 +370,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     }
     fence_proxy_async();
     tc_fence_before();
+    if (!q_ready) {   // the query image must have landed before the first MMA reads it
+      ok = __syncthreads_and(mbar_wait(bar_q, 0)) != 0;
+      q_ready = true;
+      if (!ok) break;
+    }
     __syncthreads();
 
     // ---- S^T = X . Q~^T

@@ -129,6 +129,8 @@ int make_params(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int batc
   q.table_stride = cache->table_stride;
   q.comp_blocks = cache->comp_blocks;
   q.win_blocks = cfg->window > 0 ? cache->win_blocks : 0;
+  for (int i = 0; i < LayerParams::kRopeTable; ++i)
+    q.inv_freq[i] = i < q.d_r / 2 ? std::pow(q.rope_base, -(2.0 * i) / static_cast<double>(q.d_r)) : 0.0;
   return CKV_OK;
 }
 

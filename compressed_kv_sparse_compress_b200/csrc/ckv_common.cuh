@@ -34,6 +34,10 @@ struct LayerParams {
   const int32_t* win_table;
   int table_stride;
   int comp_blocks, win_blocks;
+  // base^(-2i/d_r) for rotary pair i, computed on the host in fp64 (d_r <= 2 * kRopeTable;
+  // larger rotary widths compute it on the device)
+  static constexpr int kRopeTable = 64;
+  double inv_freq[kRopeTable];
 };
 
 // ------------------------------------------------------------------------------- formats
@@ -70,6 +74,11 @@ __device__ __forceinline__ __half2 e2m1x2_to_half2(uint8_t byte) {
 // inverse frequency of rotary pair i: base^(-2i/d_r), fp64
 __device__ __forceinline__ double rope_inv_freq(int i, int d_r, double base) {
   return pow(base, -(2.0 * i) / static_cast<double>(d_r));
+}
+
+// the same, from the layer's host-computed table when it holds pair i
+__device__ __forceinline__ double rope_inv_freq(const LayerParams& p, int i) {
+  return i < LayerParams::kRopeTable ? p.inv_freq[i] : rope_inv_freq(i, p.d_r, p.rope_base);
 }
 
 // rotate the pair (a, b) by angle pos * inv_freq (inverse: by the negative angle), in fp64

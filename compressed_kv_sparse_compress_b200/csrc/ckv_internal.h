@@ -71,12 +71,16 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
 
 // ---------------------------------------------------------------------------- attention
 struct AttnWs {
-  float* part_o;   // [B][S][H][D]   un-normalised partial outputs
-  float* part_ml;  // [B][S][H][2]   running max and sum of each split
-  int splits;      // S: splits per request
+  float* part_o;     // [B][S][H][D]   un-normalised partial outputs
+  float* part_ml;    // [B][S][H][2]   running max and sum of each split
+  double* rope;      // [B][d_r/2][2]  cos, sin of each rotary pair at the query position
+  uint8_t* qimage;   // [B][H*D*2]     tensor-core path: rotated fp16 query in the swizzled
+                     //                shared-memory layout of the MMA operand
+  int splits;        // S: splits per request
   int keys_per_split;
   size_t bytes;
 };
+constexpr int kQImageBytes = 64 * 512 * 2;  // H = 64, D = 512 fp16
 AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len,
                            int max_selected);
 

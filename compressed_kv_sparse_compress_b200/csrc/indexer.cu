@@ -154,11 +154,17 @@ __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const
     double s0 = 0.0, s1 = 0.0;
     if (pr < npairs) {
       const int h_lo = (p.H * qtr) / 4, h_hi = (p.H * (qtr + 1)) / 4;
-#pragma unroll 16
-      for (int h = h_lo; h < h_hi; ++h) {
-        const float2 v = __ldg(reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h) * p.D) + pr);
-        s0 += v.x;
-        s1 += v.y;
+      for (int h0 = h_lo; h0 < h_hi; h0 += 16) {   // sixteen loads in flight, then the sums
+        float2 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          v[u] = h0 + u < h_hi ? __ldg(reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h0 + u) * p.D) + pr)
+                               : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          s0 += v[u].x;
+          s1 += v[u].y;
+        }
       }
     }
     part[qtr][0][threadIdx.x & 255] = s0;
@@ -170,7 +176,7 @@ __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const
       s1 = (part[0][1][k] + part[1][1][k]) + (part[2][1][k] + part[3][1][k]);
       if (pr >= first_rope && ok)
         rope_rotate_pair(s0, s1, static_cast<double>(L - 1),
-                         rope_inv_freq(pr - first_rope, p.d_r, p.rope_base), false, &s0, &s1);
+                         rope_inv_freq(p, pr - first_rope), false, &s0, &s1);
       reinterpret_cast<float2*>(ws.qbar + static_cast<int64_t>(b) * p.D)[pr] =
           make_float2(static_cast<float>(s0 * scale), static_cast<float>(s1 * scale));
     }
@@ -223,7 +229,7 @@ __device__ __forceinline__ float vec_dot(const float* qv, uint4 raw, uint32_t sc
 
 // NV: 16-byte code vectors per entry (a power of two); U: entries per lane group per chunk
 template <int DT, int NV, int U>
-__global__ void __launch_bounds__(kThreads) score_kernel(LayerParams p, int batch, IndexerWs ws,
+__global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int batch, IndexerWs ws,
                                                          float* scores, int64_t stride,
                                                          uint32_t* status) {
   griddep_wait();
@@ -265,16 +271,38 @@ __global__ void __launch_bounds__(kThreads) score_kernel(LayerParams p, int batc
   const int sub = lane % LPE, slot = lane / LPE;
   const int sc_bytes = p.D / 16;
 
-  int cur_b = -1;
-  float qreg[VPL][EPV];
-  for (int64_t ch = c_lo + warp; ch < c_hi; ch += kWarps) {
-    // request of this chunk: last b with chunk_prefix[b] <= ch
-    int lo = 0, hi = batch;
+  // A chunk's request, first entry and pool rows; resolving the next chunk (its block-table
+  // loads) overlaps the data loads of the current one.
+  struct Chunk {
+    int b;
+    int N;
+    int64_t e_base;
+    int64_t row[U];
+  };
+  auto resolve = [&](int64_t ch) {
+    Chunk c;
+    int lo = 0, hi = batch;   // last b with chunk_prefix[b] <= ch
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (chunk_prefix[mid] <= ch) lo = mid; else hi = mid;
     }
-    const int b = lo;
+    c.b = lo;
+    c.N = ws.n_c[lo];
+    c.e_base = (ch - chunk_prefix[lo]) * CH;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t e = c.e_base + u * EPP + slot;
+      c.row[u] = e < c.N ? comp_row(p, lo, e, status) : -1;
+    }
+    return c;
+  };
+
+  int cur_b = -1;
+  float qreg[VPL][EPV];
+  Chunk cur;
+  if (c_lo + warp < c_hi) cur = resolve(c_lo + warp);
+  for (int64_t ch = c_lo + warp; ch < c_hi; ch += kWarps) {
+    const int b = cur.b;
     if (b != cur_b) {
       const float* qb = ws.qbar + static_cast<int64_t>(b) * p.D;
 #pragma unroll
@@ -287,15 +315,13 @@ __global__ void __launch_bounds__(kThreads) score_kernel(LayerParams p, int batc
       }
       cur_b = b;
     }
-    const int N = ws.n_c[b];
-    const int64_t e_base = (ch - chunk_prefix[b]) * CH;
+    const int N = cur.N;
+    const int64_t e_base = cur.e_base;
     uint4 raw[U][VPL];
     uint32_t sc[U][VPL];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t e = e_base + u * EPP + slot;
-      int64_t row = -1;
-      if (e < N) row = comp_row(p, b, e, status);
+      const int64_t row = cur.row[u];
 #pragma unroll
       for (int k = 0; k < VPL; ++k) {
         const int v = sub + LPE * k;
@@ -310,6 +336,7 @@ __global__ void __launch_bounds__(kThreads) score_kernel(LayerParams p, int batc
         }
       }
     }
+    if (ch + kWarps < c_hi) cur = resolve(ch + kWarps);
     float acc[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -336,6 +363,7 @@ __global__ void __launch_bounds__(kThreads) score_kernel(LayerParams p, int batc
       atomicAdd(ws.hist + static_cast<int64_t>(b) * kHistBins + bin, static_cast<uint32_t>(__popc(same)));
   }
 }
+
 
 // ---------------------------------------------------------------------------- selection
 
@@ -539,11 +567,13 @@ cudaError_t dispatch_score(const LayerParams& p, int batch, int max_seq_len, con
   // 16-byte vectors per entry for D = 64 .. 1024: f32 D/4, bf16 D/8, nvfp4 D/32
   const int nv = p.comp_row_bytes / 16;
   constexpr int kMin = DT == CKV_F32 ? 16 : DT == CKV_BF16 ? 8 : 2;
+// entries per lane group and chunk: 8, fewer when an entry spans more than 64 vectors (the raw
+// registers of a chunk stay at 16 vectors per lane)
 #define CKV_SCORE_CASE(M)                                                                    \
   case kMin * M:                                                                             \
-    return launch_score<DT, kMin * M, (kMin * M < 8 ? kMin * M : 8)>(p, batch, max_seq_len,  \
-                                                                    ws, scores, stride,      \
-                                                                    status, stream);
+    return launch_score<DT, kMin * M,                                                        \
+                        (kMin * M < 8 ? kMin * M : (kMin * M > 64 ? 512 / (kMin * M) : 8))>( \
+        p, batch, max_seq_len, ws, scores, stride, status, stream);
   switch (nv) {
     CKV_SCORE_CASE(1)
     CKV_SCORE_CASE(2)

@@ -94,6 +94,14 @@ def csa_b4_ctx1m() -> Workload:
                     "top-k 2048, 128-token FP8 window, bf16 compressed cache, paged")
 
 
+def csa_b4_ctx256k() -> Workload:
+    return Workload(
+        "csa_b4_ctx256k_h64_d512_bf16_fp8win", (262144,) * 4, 64, 512, 64, 128,
+        (LayerSpec(4, 2048, "bf16", "fp8"),), paged=True, from_scratch=False, seed=1006,
+        description="1 CSA layer, batch 4, context 262144, H=64, D=512, r=4 (65536 entries, 256 MiB "
+                    "of keys: larger than L2), top-k 2048, FP8 window, bf16 compressed cache, paged")
+
+
 def mixed_lengths(seed: int = 1005, n: int = 64) -> tuple:
     rng = np.random.Generator(np.random.PCG64(seed))
     prev = np.clip(np.rint(np.exp(rng.normal(math.log(16384.0), 1.0, size=n))), 1024, 524288)
@@ -115,6 +123,7 @@ WORKLOADS = {
     "csa_b8_ctx32k": csa_b8_ctx32k,
     "hca_b32_ctx128k": hca_b32_ctx128k,
     "csa_b4_ctx1m": csa_b4_ctx1m,
+    "csa_b4_ctx256k": csa_b4_ctx256k,
     "mixed_64req": mixed_64req,
 }
 
