@@ -37,7 +37,7 @@ EXPORTS = (
     "kv_block_pool_num_free", "ckv_cache_row_bytes", "ckv_score_stride",
     "ckv_indexer_workspace_bytes", "ckv_attention_workspace_bytes", "kv_compress_append",
     "sparse_indexer_topk", "compressed_window_attention", "ckv_status_str", "ckv_launch_count",
-    "ckv_profile_events",
+    "ckv_profile_events", "sparse_indexer_topk_noalloc",
 )
 CKV_PROF_SCORE, CKV_PROF_ATTENTION = 0, 1
 
@@ -98,6 +98,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                         vp, vp, vp, sz, vp, vp]
     lib.compressed_window_attention.argtypes = [P(LayerCfgC), P(LayerCacheC), i32, vp, i32, vp,
                                                 vp, vp, i32, vp, vp, sz, vp, vp]
+    lib.sparse_indexer_topk_noalloc.argtypes = [P(LayerCfgC), P(LayerCacheC), i32, vp, i32, vp, i32,
+                                                vp, vp, vp, vp, vp]
+    lib.sparse_indexer_topk_noalloc.restype = ctypes.c_int
     lib.ckv_status_str.argtypes = [ctypes.c_int]
     lib.ckv_status_str.restype = ctypes.c_char_p
     lib.ckv_profile_events.argtypes = [ctypes.c_int, vp, vp]
@@ -275,6 +278,17 @@ def sparse_indexer_topk(cfg: LayerConfig, cache: LayerCache, seq_len: torch.Tens
         ctypes.byref(cfg.c()), ctypes.byref(cache.c()), batch, _ptr(seq_len), max_seq_len, _ptr(q),
         top_k, _ptr(idx), _ptr(cnt), _ptr(scores), _ptr(workspace), workspace.numel(),
         _ptr(status), _stream(stream)))
+
+
+def sparse_indexer_topk_noalloc(cfg: LayerConfig, cache: LayerCache, seq_len: torch.Tensor,
+                                max_seq_len: int, q: torch.Tensor, top_k: int, idx: torch.Tensor,
+                                cnt: torch.Tensor, status: torch.Tensor,
+                                scores: torch.Tensor | None = None, stream=None) -> None:
+    """sparse_indexer_topk with the library's own fixed scratch (no workspace, no allocation)."""
+    batch = int(seq_len.shape[0])
+    _check("sparse_indexer_topk_noalloc", load_library().sparse_indexer_topk_noalloc(
+        ctypes.byref(cfg.c()), ctypes.byref(cache.c()), batch, _ptr(seq_len), max_seq_len, _ptr(q),
+        top_k, _ptr(idx), _ptr(cnt), _ptr(scores), _ptr(status), _stream(stream)))
 
 
 def compressed_window_attention(cfg: LayerConfig, cache: LayerCache, seq_len: torch.Tensor,

@@ -222,6 +222,27 @@ int compressed_window_attention(const ckv_layer_cfg* cfg, const ckv_layer_cache*
                                 uint32_t* d_status, void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* sparse_indexer_topk without a caller-allocated workspace. The pages have no counterpart to
+ * this entry point; it exists for callers that cannot allocate device memory (an extension
+ * inside a host program that owns all device memory and gives extensions no allocator, or a
+ * latency-critical path where an allocation would synchronize the device).
+ *
+ * Same arguments, results and errors as sparse_indexer_topk minus d_ws / ws_bytes: the scratch
+ * comes from a 16 MiB array owned by the library, which every GPU that loads the library holds
+ * until the process exits. Sizes whose ckv_indexer_workspace_bytes() exceeds 16 MiB return
+ * CKV_ERR_WORKSPACE before anything is enqueued. No allocation of any kind is made.
+ *
+ * The first call on a device looks up the array's device address on that device (a host-side
+ * runtime query, no allocation); make that first call before any stream capture. All calls share
+ * the array and it keeps the last call's contents: the kernels reset the parts that must start at
+ * zero on every call, and calls whose kernels overlap on the GPU (other streams, or unordered
+ * threads) race on it. */
+int sparse_indexer_topk_noalloc(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache,
+                                int32_t batch, const int32_t* d_seq_len, int32_t max_seq_len,
+                                const float* d_q, int32_t top_k, int32_t* d_idx, int32_t* d_cnt,
+                                float* d_scores, uint32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
 /* Diagnostics. */
 
 /* Static text of a ckv_status. */
