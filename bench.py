@@ -85,6 +85,20 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(x: float, device="cpu") -> float:
+    """The largest value of x over all ranks (x itself without a process group)."""
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized() and \
+            torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step: int, world: int, steps: int, max_total_ms: float) -> float:
+    """Whole-job rate: the units every rank processed in `steps` steps over the slowest rank's time."""
+    return units_per_rank_step * world * steps / (max_total_ms / 1e3)
+
+
 def measured_peak():
     try:
         with open(PEAKS_FILE) as f:
@@ -276,11 +290,7 @@ def run_cuda(args, w: S.Workload):
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     dom_ms = [a.elapsed_time(b) for row in kev for a, b in row]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     if step.status() != 0:
         raise RuntimeError(f"device status {step.status():#x} in the timed region")
 
@@ -318,14 +328,10 @@ def run_cuda(args, w: S.Workload):
         e2e_step()
         eev[i][1].record(stream)
     barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev), dev)
 
     units = w.batch * len(w.layers) * ws  # queries*layers per step over all ranks
-    value = units * args.steps / (total_ms / 1e3)
+    value = job_throughput(w.batch * len(w.layers), ws, args.steps, total_ms)
     peak, peak_src = measured_peak()
     lb = [layer_bytes(w, ls) for ls in w.layers]
     if dominant == "score_kernel":
@@ -358,7 +364,7 @@ def run_cuda(args, w: S.Workload):
                      "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
                      "avg_launch_us": dom_avg_ms * 1e3, "algorithmic_bytes": dom_bytes,
                      "traffic": traffic_record(dominant, w.name)},
-        "e2e": {"value": units * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": job_throughput(w.batch * len(w.layers), ws, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": launches,

@@ -114,6 +114,42 @@ __device__ void store_entry(const LayerParams& p, int64_t row, const float* c) {
   }
 }
 
+// Weighted sum of ring tokens [t0, t0 + n_ring) of one group, split across the CTA's warps: warp w
+// takes a contiguous run of tokens, lane l the rotary-aligned pairs l + 32k (NPL of them), BT
+// tokens' loads in flight; each warp writes its partial sums to part[w][D] (zeros if it has none).
+template <int NPL, int BT>
+__device__ void ring_partial(const float* ring, const float* w, int64_t t0, int r, int n_ring,
+                             float* part) {
+  constexpr int D = 64 * NPL;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int per = (n_ring + nw - 1) / nw;
+  const int tlo = warp * per, thi = min(n_ring, tlo + per);
+  float2 acc[NPL];
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) acc[k] = make_float2(0.f, 0.f);
+  for (int tb = tlo; tb < thi; tb += BT) {
+    float2 x[BT][NPL];
+#pragma unroll
+    for (int u = 0; u < BT; ++u) {
+      const int t = tb + u;
+      const float2* row = reinterpret_cast<const float2*>(ring + ((t0 + t) % r) * D);
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) x[u][k] = t < thi ? row[lane + 32 * k] : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < BT; ++u) {
+      const float wt = tb + u < thi ? w[tb + u] : 0.f;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        acc[k].x = fmaf(wt, x[u][k].x, acc[k].x);
+        acc[k].y = fmaf(wt, x[u][k].y, acc[k].y);
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) reinterpret_cast<float2*>(part + warp * D)[lane + 32 * k] = acc[k];
+}
+
 // Handles group g of request b: writes the new tokens' window / ring slots and, when the group
 // is complete, folds it into entry g.
 __device__ void process_group(const AppendArgs& a, int b, int64_t g, int64_t prev, int64_t new_len,
@@ -178,26 +214,32 @@ __device__ void process_group(const AppendArgs& a, int b, int64_t g, int64_t pre
     for (int t = threadIdx.x; t < r; t += 32) w[t] = w[t] / s;
   }
   __syncthreads();
-  // entry = sum over the group's tokens, in token order, of w_t * rotated token t
+  // entry = sum over the group's tokens of w_t * rotated token t: the tokens already in the ring
+  // are split across the warps (partial sums reduced in shared memory), then the new tokens are
+  // added in token order
+  const int64_t ring_end = min(prev, t0 + r);
+  const int n_ring = ring_end > t0 ? static_cast<int>(ring_end - t0) : 0;
+  float* part = smem + 256 + 1024 + 32;  // [warps][D]
+  switch (D) {
+    case 64: ring_partial<1, 4>(ring, w, t0, r, n_ring, part); break;
+    case 128: ring_partial<2, 4>(ring, w, t0, r, n_ring, part); break;
+    case 256: ring_partial<4, 4>(ring, w, t0, r, n_ring, part); break;
+    case 512: ring_partial<8, 4>(ring, w, t0, r, n_ring, part); break;
+    default: ring_partial<16, 2>(ring, w, t0, r, n_ring, part); break;
+  }
+  __syncthreads();
+  const int nw = blockDim.x >> 5;
   for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) {
     float2 acc = make_float2(0.f, 0.f);
-    for (int tb = 0; tb < r; tb += 4) {   // four tokens' loads in flight
-      float2 x[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t pos = t0 + tb + u;
-        if (tb + u >= r) x[u] = make_float2(0.f, 0.f);
-        else if (pos < prev) x[u] = reinterpret_cast<const float2*>(ring + (pos % r) * D)[pr];
-        else if (pos == pos_last) x[u] = xlast[k];
-        else x[u] = rotate_raw_pair(a, a.kv_new + (row0 + (pos - prev)) * D, pr, pos);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (tb + u < r) {
-          acc.x = fmaf(w[tb + u], x[u].x, acc.x);
-          acc.y = fmaf(w[tb + u], x[u].y, acc.y);
-        }
-      }
+    for (int ww = 0; ww < nw; ++ww) {
+      acc.x += part[ww * D + 2 * pr];
+      acc.y += part[ww * D + 2 * pr + 1];
+    }
+    for (int64_t pos = max(t0, prev); pos < t0 + r; ++pos) {
+      const float2 x = pos == pos_last ? xlast[k]
+                                       : rotate_raw_pair(a, a.kv_new + (row0 + (pos - prev)) * D, pr, pos);
+      acc.x = fmaf(w[pos - t0], x.x, acc.x);
+      acc.y = fmaf(w[pos - t0], x.y, acc.y);
     }
     c[2 * pr] = acc.x;
     c[2 * pr + 1] = acc.y;
@@ -210,7 +252,7 @@ __device__ void process_group(const AppendArgs& a, int b, int64_t g, int64_t pre
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
   griddep_wait();
   griddep_launch();
-  __shared__ float smem[256 + 1024 + 32];
+  __shared__ float smem[256 + 1024 + 32 + (kAppendThreads / 32) * 1024];
   const int b = blockIdx.y;
   const int64_t prev = a.prev_len[b];
   int64_t row0, n;

@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kPrepThreads) attn_prep_kernel(LayerParams p, 
   griddep_wait();
   griddep_launch();
   __shared__ double rope_s[2 * 512];
-  const int b = blockIdx.x;
+  const int b = blockIdx.y;
   const int L = seq_len[b];
   if (L < 1 || L > max_seq_len) return;
   const int n_pairs = p.d_r / 2;
@@ -180,28 +180,30 @@ __global__ void __launch_bounds__(kPrepThreads) attn_prep_kernel(LayerParams p, 
     sincos(static_cast<double>(L - 1) * rope_inv_freq(p, i), &sn, &cs);
     rope_s[2 * i] = cs;
     rope_s[2 * i + 1] = sn;
-    rope_g[2 * i] = cs;
-    rope_g[2 * i + 1] = sn;
+    if (blockIdx.x == 0) {
+      rope_g[2 * i] = cs;
+      rope_g[2 * i + 1] = sn;
+    }
   }
   if (!ws.qimage) return;
   __syncthreads();
   // tensor-core path (H = 64, D = 512): granule g (8 dims) of head h lands at chunk g/8, row h,
-  // 16-byte slot (g % 8) ^ (h % 8) of the operand image
+  // 16-byte slot (g % 8) ^ (h % 8) of the operand image; CTA x builds heads 8x .. 8x+7
   constexpr int kD = 512, kGr = kD / 8, kChunk = 64 * 128;
   const float* qb = q + static_cast<int64_t>(b) * 64 * kD;
   uint8_t* img = ws.qimage + static_cast<int64_t>(b) * kQImageBytes;
   const int first_rope = (kD - p.d_r) / 2;
-  for (int it0 = 0; it0 < 64 * kGr; it0 += 8 * kPrepThreads) {
-    float4 raw[8][2];
+  for (int it0 = blockIdx.x * 8 * kGr; it0 < (blockIdx.x + 1) * 8 * kGr; it0 += 2 * kPrepThreads) {
+    float4 raw[2][2];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int it = it0 + u * kPrepThreads + threadIdx.x;
       const float4* src = reinterpret_cast<const float4*>(qb + (it >> 6) * kD + 8 * (it & 63));
       raw[u][0] = __ldg(src);
       raw[u][1] = __ldg(src + 1);
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int it = it0 + u * kPrepThreads + threadIdx.x;
       const int h = it >> 6, g = it & 63;
       float v[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
@@ -244,66 +246,80 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(
   }
   const KeyList kl = key_list(p, L, cnt, sparse, idx_stride, b);
   const int ns = static_cast<int>((kl.n_keys + ws.keys_per_split - 1) / ws.keys_per_split);
-  // log-sum-exp merge of the splits: M = max of the split maxima, Z = sum l_s exp(m_s - M)
+  // log-sum-exp merge of the splits: M = max of the split maxima, w_s = exp(m_s - M),
+  // Z = sum_s w_s l_s; the weights of the first kCombineSmemSplits splits are kept in shared memory
+  constexpr int kCombineSmemSplits = 256;
+  __shared__ float wts[kCombineSmemSplits];
   __shared__ float red_m[32], red_z[32];
   const float2* ml = reinterpret_cast<const float2*>(ws.part_ml);
   const int64_t base = static_cast<int64_t>(b) * ws.splits;
-  float mloc = -INFINITY;
+  // one pass: each thread merges its splits' (m, l) online, then the block merges the threads
+  float mloc = -INFINITY, zloc = 0.f;
   for (int s = threadIdx.x; s < ns; s += blockDim.x) {
     const float2 v = __ldcg(ml + (base + s) * p.H + h);
-    if (v.y > 0.f) mloc = fmaxf(mloc, v.x);
+    if (s < kCombineSmemSplits) wts[s] = v.y > 0.f ? v.x : -INFINITY;
+    if (v.y > 0.f) {
+      const float mn = fmaxf(mloc, v.x);
+      zloc = zloc * expf(mloc - mn) + v.y * expf(v.x - mn);
+      mloc = mn;
+    }
   }
-  mloc = warp_max(mloc);
-  if ((threadIdx.x & 31) == 0) red_m[threadIdx.x >> 5] = mloc;
+  const float mwarp = warp_max(mloc);
+  zloc = warp_sum(mloc == -INFINITY ? 0.f : zloc * expf(mloc - mwarp));
+  if ((threadIdx.x & 31) == 0) {
+    red_m[threadIdx.x >> 5] = mwarp;
+    red_z[threadIdx.x >> 5] = zloc;
+  }
   __syncthreads();
   float M = -INFINITY;
   for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) M = fmaxf(M, red_m[i]);
-  float zloc = 0.f;
-  for (int s = threadIdx.x; s < ns; s += blockDim.x) {
-    const float2 v = __ldcg(ml + (base + s) * p.H + h);
-    if (v.y > 0.f) zloc += v.y * expf(v.x - M);
-  }
-  zloc = warp_sum(zloc);
-  if ((threadIdx.x & 31) == 0) red_z[threadIdx.x >> 5] = zloc;
-  __syncthreads();
   float Z = 0.f;
-  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) Z += red_z[i];
+  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i)
+    if (red_m[i] > -INFINITY) Z += red_z[i] * expf(red_m[i] - M);
+  // split weights exp(m_s - M) for the first kCombineSmemSplits splits
+  for (int s = threadIdx.x; s < ns && s < kCombineSmemSplits; s += blockDim.x)
+    wts[s] = wts[s] > -INFINITY ? expf(wts[s] - M) : 0.f;
+  __syncthreads();
   const float inv = Z > 0.f ? 1.f / Z : 0.f;
+  auto weight = [&](int s) -> float {
+    if (s < kCombineSmemSplits) return wts[s];
+    const float2 v = __ldcg(ml + (base + s) * p.H + h);
+    return v.y > 0.f ? expf(v.x - M) : 0.f;
+  };
   const int first_rope = (D - p.d_r) / 2;
   const double* rope = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
-  const float* po = ws.part_o + (base * p.H + h) * D;
-  const int64_t split_stride = static_cast<int64_t>(p.H) * D;
-  for (int pr = threadIdx.x; pr < D / 2; pr += blockDim.x) {
-    float2 acc = make_float2(0.f, 0.f);
+  const float4* po = reinterpret_cast<const float4*>(ws.part_o + (base * p.H + h) * D);
+  const int64_t split_stride = static_cast<int64_t>(p.H) * D / 4;
+  for (int c = threadIdx.x; c < D / 4; c += blockDim.x) {   // dims 4c .. 4c+3 (two pairs)
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = 0; s0 < ns; s0 += 8) {   // eight splits' loads in flight
       float wgt[8];
-      float2 x[8];
+      float4 x[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        wgt[u] = 0.f;
-        if (s0 + u < ns) {
-          const float2 v = __ldcg(ml + (base + s0 + u) * p.H + h);
-          if (v.y > 0.f) wgt[u] = expf(v.x - M);
-        }
-      }
+      for (int u = 0; u < 8; ++u) wgt[u] = s0 + u < ns ? weight(s0 + u) : 0.f;
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        x[u] = wgt[u] > 0.f ? __ldcg(reinterpret_cast<const float2*>(po + (s0 + u) * split_stride) + pr)
-                            : make_float2(0.f, 0.f);
+        x[u] = wgt[u] > 0.f ? __ldcg(po + (s0 + u) * split_stride + c) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         acc.x = fmaf(wgt[u], x[u].x, acc.x);
         acc.y = fmaf(wgt[u], x[u].y, acc.y);
+        acc.z = fmaf(wgt[u], x[u].z, acc.z);
+        acc.w = fmaf(wgt[u], x[u].w, acc.w);
       }
     }
-    acc.x *= inv;
-    acc.y *= inv;
-    if (pr >= first_rope) {   // inverse rotation by the query position
-      const double cs = rope[2 * (pr - first_rope)], sn = rope[2 * (pr - first_rope) + 1];
-      const double a = acc.x, c = acc.y;
-      acc = make_float2(static_cast<float>(a * cs + c * sn), static_cast<float>(c * cs - a * sn));
+    float v[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {   // inverse rotation by the query position
+      const int pr = 2 * c + k;
+      if (pr >= first_rope) {
+        const double cs = rope[2 * (pr - first_rope)], sn = rope[2 * (pr - first_rope) + 1];
+        const double a = v[2 * k], e = v[2 * k + 1];
+        v[2 * k] = static_cast<float>(a * cs + e * sn);
+        v[2 * k + 1] = static_cast<float>(e * cs - a * sn);
+      }
     }
-    reinterpret_cast<float2*>(o)[pr] = acc;
+    reinterpret_cast<float4*>(o)[c] = make_float4(v[0], v[1], v[2], v[3]);
   }
 }
 
@@ -351,7 +367,8 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
                              int max_seq_len, const float* q, const int32_t* idx,
                              const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
                              uint32_t* status, cudaStream_t stream) {
-  cudaError_t e = launch_kernel(attn_prep_kernel, dim3(batch), dim3(kPrepThreads), 0, stream, p, seq_len,
+  const dim3 prep_grid(attention_tc_supported(p) ? 8 : 1, batch);   // 8 heads per CTA on the MMA path
+  cudaError_t e = launch_kernel(attn_prep_kernel, prep_grid, dim3(kPrepThreads), 0, stream, p, seq_len,
                                 max_seq_len, q, ws);
   if (e != cudaSuccess) return e;
   prof_begin(kProfAttention, stream);

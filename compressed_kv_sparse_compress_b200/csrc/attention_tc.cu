@@ -137,6 +137,20 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n"
+               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------------ helpers
 
 __device__ __forceinline__ uint32_t half2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
@@ -150,14 +164,14 @@ __device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
   return half2_bits(__half2(r));
 }
 
-// Reduction of 64 per-thread values across a warp; afterwards t[0], t[1] hold the reduction of
-// entries 2*lane and 2*lane+1.
-template <bool kMax>
-__device__ __forceinline__ void reduce_scatter64(float (&t)[64], int lane) {
+// Reduction of N (64 or 32) per-thread values across a warp; afterwards t[0 .. N/32) hold the
+// reduction of entries (N/32)*lane .. (N/32)*lane + N/32 - 1.
+template <int N, bool kMax>
+__device__ __forceinline__ void reduce_scatter(float (&t)[N], int lane) {
 #pragma unroll
   for (int s = 0; s < 5; ++s) {
     const int o = 16 >> s;
-    const int half = 32 >> s;
+    const int half = N >> (s + 1);
     const bool upper = (lane & o) != 0;
 #pragma unroll
     for (int i = 0; i < half; ++i) {
@@ -351,21 +365,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       __syncthreads();
     }
 
-    // ---- stage the tile as fp16 (absent keys are zero rows)
+    // ---- stage the tile as fp16 (absent keys are zero rows): warp w converts keys 16w .. 16w+15,
+    //      lane l the granules l and l + 32 of each (the key's row and kind read once per key)
 #pragma unroll 1
-    for (int it0 = 0; it0 < kTile * (kD / 8); it0 += 16 * kThreads) {
-      Raw r[16];
+    for (int jb = 0; jb < 16; jb += 8) {
+      Raw r[8][2];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int it = it0 + u * kThreads + tid;
-        const int j = it >> 6, g = it & 63;
-        r[u] = load_granule<CT, WT>(p, key_row[j], key_win[j] != 0, g);
+      for (int u = 0; u < 8; ++u) {
+        const int j = 16 * warp + jb + u;
+        const int64_t row = key_row[j];
+        const bool win = key_win[j] != 0;
+        r[u][0] = load_granule<CT, WT>(p, row, win, lane);
+        r[u][1] = load_granule<CT, WT>(p, row, win, lane + 32);
       }
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int it = it0 + u * kThreads + tid;
-        const int j = it >> 6, g = it & 63;
-        st_shared_v4(sb + kOffX + swz(kXChunk, j, g), convert_granule<CT, WT>(r[u], key_win[j] != 0));
+      for (int u = 0; u < 8; ++u) {
+        const int j = 16 * warp + jb + u;
+        const bool win = key_win[j] != 0;
+        st_shared_v4(sb + kOffX + swz(kXChunk, j, lane), convert_granule<CT, WT>(r[u][0], win));
+        st_shared_v4(sb + kOffX + swz(kXChunk, j, lane + 32), convert_granule<CT, WT>(r[u][1], win));
       }
     }
     fence_proxy_async();
@@ -396,22 +414,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     tc_fence_after();
     if (!ok) break;
 
-    // ---- softmax over the tile's keys (warps 0-3: thread = key = TMEM lane)
-    if (warp < 4) {
-      uint32_t raw[64];
-      tmem_ld64(tmem + (static_cast<uint32_t>(warp * 32) << 16) + kSCol, raw);
-      const float f = key_ls[tid];
-      const bool valid = key_row[tid] >= 0;
-      float sv[64], t[64];
+    // ---- softmax over the tile's keys: key j = TMEM lane; warp w reads the lanes of quarter w%4
+    //      and the 32 heads of half w/4
+    {
+      const int q4 = warp & 3, half = warp >> 2;
+      const int j = q4 * 32 + lane;
+      const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+      uint32_t raw[32];
+      tmem_ld32(tmem + lane_base + kSCol + 32 * half, raw);
+      const float f = key_ls[j];
+      const bool valid = key_row[j] >= 0;
+      float sv[32], t[32];
 #pragma unroll
-      for (int h = 0; h < 64; ++h) {
+      for (int h = 0; h < 32; ++h) {
         sv[h] = valid ? __uint_as_float(raw[h]) * f : -INFINITY;
         t[h] = sv[h];
       }
-      reduce_scatter64<true>(t, lane);
-      red[warp * kH + 2 * lane] = t[0];
-      red[warp * kH + 2 * lane + 1] = t[1];
-      named_sync(1, 128);
+      reduce_scatter<32, true>(t, lane);
+      red[q4 * kH + 32 * half + lane] = t[0];
+      __syncthreads();
       if (tid < kH) {
         const float mt = fmaxf(fmaxf(red[tid], red[kH + tid]), fmaxf(red[2 * kH + tid], red[3 * kH + tid]));
         const float mo = m_run[tid];
@@ -424,12 +445,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         m_run[tid] = mn;
         alpha[tid] = al;
       }
-      named_sync(1, 128);
-      const float vs = key_vs[tid];
-      uint32_t packed[32];
+      __syncthreads();
+      const float vs = key_vs[j];
+      uint32_t packed[16];
 #pragma unroll
-      for (int h = 0; h < 64; h += 2) {
-        const float m0 = m_run[h], m1 = m_run[h + 1];
+      for (int h = 0; h < 32; h += 2) {
+        const float m0 = m_run[32 * half + h], m1 = m_run[32 * half + h + 1];
         const float p0 = m0 == -INFINITY ? 0.f : __expf(sv[h] - m0);
         const float p1 = m1 == -INFINITY ? 0.f : __expf(sv[h + 1] - m1);
         t[h] = p0;
@@ -437,25 +458,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         packed[h >> 1] = pack_f32x2(p0 * vs, p1 * vs);
       }
 #pragma unroll
-      for (int g = 0; g < 8; ++g)
-        st_shared_v4(sb + kOffP + static_cast<uint32_t>(tid) * 128u + (static_cast<uint32_t>(g ^ (tid & 7)) << 4),
+      for (int g = 0; g < 4; ++g)
+        st_shared_v4(sb + kOffP + static_cast<uint32_t>(j) * 128u +
+                         (static_cast<uint32_t>((4 * half + g) ^ (j & 7)) << 4),
                      make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]));
-      reduce_scatter64<false>(t, lane);
-      red[warp * kH + 2 * lane] = t[0];
-      red[warp * kH + 2 * lane + 1] = t[1];
-      named_sync(1, 128);
+      reduce_scatter<32, false>(t, lane);
+      red[q4 * kH + 32 * half + lane] = t[0];
+      __syncthreads();
       if (tid < kH)
         l_run[tid] = l_run[tid] * alpha[tid] + ((red[tid] + red[kH + tid]) + (red[2 * kH + tid] + red[3 * kH + tid]));
       // rescale the output accumulated so far where the running max was raised
       if (tile > 0 && flags[0]) {
 #pragma unroll 1
         for (int m = 0; m < 4; ++m) {
-          const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16) + kOCol + 64 * m;
-          uint32_t o[64];
-          tmem_ld64(ta, o);
+          const uint32_t ta = tmem + lane_base + kOCol + 64 * m + 32 * half;
+          uint32_t o[32];
+          tmem_ld32(ta, o);
 #pragma unroll
-          for (int h = 0; h < 64; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-          tmem_st64(ta, o);
+          for (int h = 0; h < 32; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[32 * half + h]);
+          tmem_st32(ta, o);
         }
       }
       fence_proxy_async();
@@ -468,11 +489,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     if (tid == 128) {
       tc_fence_after();
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
+      for (int kk = 0; kk < kTile / 16; ++kk) {   // consecutive MMAs go to different accumulators
+        const uint64_t bp = sdesc(sb + kOffP + kk * 2048, 8192, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
+        for (int m = 0; m < 4; ++m) {
           const uint64_t a = sdesc(sb + kOffX + 2 * m * kXChunk + kk * 2048, kXChunk, 1024);
-          const uint64_t bp = sdesc(sb + kOffP + kk * 2048, 8192, 1024);
           mma_f16(tmem + kOCol + 64 * m, a, bp, kIdescPV, (tile > 0 || kk > 0) ? 1u : 0u);
         }
       }
@@ -483,25 +504,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     tc_fence_after();
   }
 
-  // ---- partial outputs: O^T lane = dim, column = head
-  if (ok && warp < 4) {
+  // ---- partial outputs: O^T lane = dim, column = head (warp w: lane quarter w%4, heads of half w/4)
+  if (ok) {
+    const int q4 = warp & 3, half = warp >> 2;
     const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
 #pragma unroll 1
     for (int m = 0; m < 4; ++m) {
-      uint32_t o[64];
-      tmem_ld64(tmem + (static_cast<uint32_t>(warp * 32) << 16) + kOCol + 64 * m, o);
-      const int d = 128 * m + tid;
+      uint32_t o[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + kOCol + 64 * m + 32 * half, o);
+      const int d = 128 * m + 32 * q4 + lane;
 #pragma unroll
-      for (int h = 0; h < 64; ++h) ws.part_o[(slot + h) * kD + d] = __uint_as_float(o[h]);
+      for (int h = 0; h < 32; ++h) ws.part_o[(slot + 32 * half + h) * kD + d] = __uint_as_float(o[h]);
     }
     if (tid < kH) reinterpret_cast<float2*>(ws.part_ml)[slot + tid] = make_float2(m_run[tid], l_run[tid]);
   }
   if (!ok) {
     if (tid == 0) atomicOr(status, CKV_DEV_TIMEOUT);
-    if (warp < 4) {
-      const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
-      if (tid < kH) reinterpret_cast<float2*>(ws.part_ml)[slot + tid] = make_float2(-INFINITY, 0.f);
-    }
+    const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
+    if (tid < kH) reinterpret_cast<float2*>(ws.part_ml)[slot + tid] = make_float2(-INFINITY, 0.f);
   }
   tc_fence_before();
   __syncthreads();

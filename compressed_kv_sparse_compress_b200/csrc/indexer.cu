@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const
   const double scale = static_cast<double>(p.sm_scale) / p.H;
   for (int pr0 = 0; pr0 < npairs; pr0 += 256) {   // D <= 1024: at most two rounds
     const int pr = pr0 + (threadIdx.x & 255), qtr = threadIdx.x >> 8;
-    double s0 = 0.0, s1 = 0.0;
+    double s0 = 0.0, s1 = 0.0, rsn = 0.0, rcs = 1.0;
     if (pr < npairs) {
       const int h_lo = (p.H * qtr) / 4, h_hi = (p.H * (qtr + 1)) / 4;
       for (int h0 = h_lo; h0 < h_hi; h0 += 16) {   // sixteen loads in flight, then the sums
@@ -160,6 +160,8 @@ __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const
         for (int u = 0; u < 16; ++u)
           v[u] = h0 + u < h_hi ? __ldg(reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h0 + u) * p.D) + pr)
                                : make_float2(0.f, 0.f);
+        if (h0 == h_lo && qtr == 0 && pr >= first_rope && ok)   // rotation angle while loads fly
+          sincos(static_cast<double>(L - 1) * rope_inv_freq(p, pr - first_rope), &rsn, &rcs);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           s0 += v[u].x;
@@ -174,9 +176,11 @@ __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const
       const int k = threadIdx.x & 255;
       s0 = (part[0][0][k] + part[1][0][k]) + (part[2][0][k] + part[3][0][k]);
       s1 = (part[0][1][k] + part[1][1][k]) + (part[2][1][k] + part[3][1][k]);
-      if (pr >= first_rope && ok)
-        rope_rotate_pair(s0, s1, static_cast<double>(L - 1),
-                         rope_inv_freq(p, pr - first_rope), false, &s0, &s1);
+      if (pr >= first_rope && ok) {
+        const double a = s0, c = s1;
+        s0 = a * rcs - c * rsn;
+        s1 = a * rsn + c * rcs;
+      }
       reinterpret_cast<float2*>(ws.qbar + static_cast<int64_t>(b) * p.D)[pr] =
           make_float2(static_cast<float>(s0 * scale), static_cast<float>(s1 * scale));
     }
@@ -539,6 +543,95 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, 
   if (threadIdx.x == 0) cnt[b] = static_cast<int32_t>(k_eff);
 }
 
+
+// Whole selection of one request in one CTA, for up to kSmallPerThread * 512 candidates: the
+// scores stay in registers (thread t holds a contiguous run of indices), three radix digits are
+// counted in shared memory, ties at the threshold key go to the lowest indices through a block
+// scan in index order, and the winners are written in ascending order by a second block scan.
+constexpr int kSmallThreads = 512;
+constexpr int kSmallPerThread = 32;
+constexpr int kSmallMax = kSmallThreads * kSmallPerThread;
+
+__global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* scores, int64_t stride,
+                                                                   int top_k, IndexerWs ws,
+                                                                   int32_t* idx, int32_t* cnt) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ uint32_t h[kHistBins];
+  __shared__ uint32_t sh[32];
+  __shared__ uint32_t bnd[2];
+  const int b = blockIdx.x;
+  const int N = ws.n_c[b];
+  const int k_eff = N < top_k ? N : top_k;
+  const int per = (N + kSmallThreads - 1) / kSmallThreads;
+  const int j0 = threadIdx.x * per;
+  int32_t* out = idx + static_cast<int64_t>(b) * top_k;
+  uint32_t key[kSmallPerThread];
+  const float* sb = scores + static_cast<int64_t>(b) * stride;
+#pragma unroll
+  for (int u = 0; u < kSmallPerThread; ++u) key[u] = (u < per && j0 + u < N) ? f32_order_key(__ldcg(sb + j0 + u)) : 0u;
+
+  uint32_t T = 0, idx_quota = 0;  // selected: key > T, or key == T among the first idx_quota
+  bool all = N <= top_k;
+  if (!all) {
+    uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k_eff);
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+      const int shift = d == 0 ? 21 : (d == 1 ? 10 : 0);
+      const int nb = d == 2 ? 1024 : 2048;
+      if (d == 0) {
+        // the first digit was counted by the score kernel
+        for (int i = threadIdx.x; i < nb; i += blockDim.x) h[i] = __ldcg(ws.hist + static_cast<int64_t>(b) * kHistBins + i);
+      } else {
+        for (int i = threadIdx.x; i < nb; i += blockDim.x) h[i] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kSmallPerThread; ++u)   // only keys in the boundary bin so far
+          if (u < per && j0 + u < N && (key[u] & mask) == prefix)
+            atomicAdd(h + ((key[u] >> shift) & (nb - 1)), 1u);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) bnd[0] = bnd[1] = 0;
+      find_boundary(h, nb, need, true, sh, bnd);
+      need -= bnd[1];
+      prefix |= bnd[0] << shift;
+      mask |= static_cast<uint32_t>(nb - 1) << shift;
+      __syncthreads();
+    }
+    T = prefix;
+    idx_quota = need;   // how many of the key == T candidates are taken, lowest indices first
+  }
+  // rank of each key == T among equals in index order
+  uint32_t n_eq = 0;
+#pragma unroll
+  for (int u = 0; u < kSmallPerThread; ++u)
+    if (!all && u < per && j0 + u < N && key[u] == T) ++n_eq;
+  const uint32_t eq_incl = block_inclusive_scan<uint32_t>(n_eq, sh, nullptr);
+  uint32_t eq_rank = eq_incl - n_eq;
+  uint32_t sel_mask = 0, n_sel = 0;
+#pragma unroll
+  for (int u = 0; u < kSmallPerThread; ++u) {
+    if (u < per && j0 + u < N) {
+      bool take = all || key[u] > T;
+      if (!all && key[u] == T) take = eq_rank++ < idx_quota;
+      if (take) {
+        sel_mask |= 1u << u;
+        ++n_sel;
+      }
+    }
+  }
+  const uint32_t sel_incl = block_inclusive_scan<uint32_t>(n_sel, sh, nullptr);
+  uint32_t pos = sel_incl - n_sel;
+#pragma unroll
+  for (int u = 0; u < kSmallPerThread; ++u)
+    if (sel_mask & (1u << u)) {
+      if (pos < static_cast<uint32_t>(top_k)) out[pos] = j0 + u;
+      ++pos;
+    }
+  for (int i = k_eff + threadIdx.x; i < top_k; i += blockDim.x) out[i] = -1;
+  if (threadIdx.x == 0) cnt[b] = k_eff;
+}
+
 template <int DT, int NV, int U>
 cudaError_t launch_score(const LayerParams& p, int batch, int max_seq_len, const IndexerWs& ws,
                          float* scores, int64_t stride, uint32_t* status, cudaStream_t stream) {
@@ -546,14 +639,18 @@ cudaError_t launch_score(const LayerParams& p, int batch, int max_seq_len, const
   constexpr int CH = U * (32 / LPE);
   const int64_t per_req = (static_cast<int64_t>(max_seq_len) / p.r + CH - 1) / CH;
   const int64_t chunks = per_req * batch;
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 4 * kWarps;  // warps resident
-  int64_t grid = (chunks + kWarps - 1) / kWarps;
-  if (grid > cap / kWarps) grid = cap / kWarps;
-  if (grid < 1) grid = 1;
   const int smem = static_cast<int>(sizeof(int32_t) * (batch + 1));
   auto kern = score_kernel<DT, NV, U>;
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
+  // one wave of persistent CTAs: as many as fit on every SM at once
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  int64_t grid = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
+  const int64_t useful = (chunks + kWarps - 1) / kWarps;
+  if (grid > useful) grid = useful;
+  if (grid < 1) grid = 1;
   prof_begin(kProfScore, stream);
   e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, p, batch, ws,
                     scores, stride, status);
@@ -605,6 +702,9 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
   }
   if (e != cudaSuccess) return e;
   const int64_t nmax = static_cast<int64_t>(max_seq_len) / p.r;
+  if (nmax <= kSmallMax)   // every request's candidates fit one CTA's registers
+    return launch_kernel(topk_small_kernel, dim3(batch), dim3(kSmallThreads), 0, stream,
+                         static_cast<const float*>(sc), stride, top_k, ws, idx, cnt);
   dim3 mgrid(static_cast<unsigned>(nmax > 0 ? (nmax + kMarkChunk - 1) / kMarkChunk : 1), batch);
   e = launch_kernel(topk_mark_kernel, mgrid, dim3(kThreads), 0, stream, static_cast<const float*>(sc),
                     stride, top_k, ws);
