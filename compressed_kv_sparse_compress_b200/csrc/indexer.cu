@@ -9,10 +9,13 @@
 // per request, and scoring streams the compressed cache once with one fp32 dot per entry.
 //
 // Kernels, in stream order:
-//   qbar_kernel     per request: q_bar, candidate count, reset of the selection state
+//   qbar_kernel     per (request, slice of dims): q_bar, candidate count, reset of the
+//                   selection state
 //   score_kernel    persistent, HBM-bound: streams every candidate entry with 16-byte
 //                   non-allocating loads, writes its fp32 score, and counts the top 11 bits of
 //                   its order key into a per-request histogram (first radix digit)
+//   topk_small      per request, when every request has at most 16384 candidates: the whole
+//                   selection in one CTA with the scores in registers
 //   topk_mark       per (request, 8192 scores): marks scores above the boundary bin in a
 //                   bitmap and appends boundary-bin candidates to a list
 //   topk_finish     per request: resolves the boundary bin with two more radix digits (and the
@@ -127,64 +130,74 @@ __device__ void find_boundary(const uint32_t* h, int nbins, uint32_t need, bool 
 
 // ---------------------------------------------------------------------------- q_bar
 
-// One CTA of 1024 threads per request: thread (pair, quarter) sums a quarter of the heads of one
-// rotary-aligned pair of dims in fp64; the quarters are added in shared memory.
-constexpr int kQbarThreads = 1024;
+// kQbarSlices CTAs of 256 threads per request, CTA s owning the rotary-aligned dim pairs
+// [s * P, (s + 1) * P) with P = D / 2 / kQbarSlices: thread (pair k, head group g) sums its heads of
+// one pair in fp64 with all its loads in flight at once; the head groups are added in shared
+// memory, the sum rotated and scaled. The slices also reset the request's selection state.
+constexpr int kQbarThreads = 256;
+constexpr int kQbarSlices = 8;
 
 __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const int32_t* seq_len,
                                                             int max_seq_len, const float* q,
                                                             IndexerWs ws, uint32_t* status) {
   griddep_wait();
   griddep_launch();
-  __shared__ double part[4][2][256];
-  const int b = blockIdx.x;
+  __shared__ double part[kQbarThreads][2];
+  const int b = blockIdx.y, slice = blockIdx.x, tid = threadIdx.x;
   const int L = seq_len[b];
   const bool ok = L >= 1 && L <= max_seq_len;
-  if (threadIdx.x == 0) {
+  if (slice == 0 && tid == 0) {
     if (!ok) atomicOr(status, CKV_DEV_BAD_LENGTH);
     ws.n_c[b] = ok ? L / p.r : 0;
     ws.cand_cnt[b] = 0;
   }
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ws.hist[static_cast<int64_t>(b) * kHistBins + i] = 0;
-  const int npairs = p.D / 2, first_rope = (p.D - p.d_r) / 2;
+  constexpr int kBinsPerSlice = kHistBins / kQbarSlices;
+  for (int i = tid; i < kBinsPerSlice; i += kQbarThreads)
+    ws.hist[static_cast<int64_t>(b) * kHistBins + slice * kBinsPerSlice + i] = 0;
+  const int P = p.D / 2 / kQbarSlices;  // 4 .. 64 pairs (D = 64 .. 1024)
+  const int G = kQbarThreads / P;       // head groups
+  const int k = tid % P, g = tid / P;
+  const int pr = slice * P + k, first_rope = (p.D - p.d_r) / 2;
   const float* qb = q + static_cast<int64_t>(b) * p.H * p.D;
-  const double scale = static_cast<double>(p.sm_scale) / p.H;
-  for (int pr0 = 0; pr0 < npairs; pr0 += 256) {   // D <= 1024: at most two rounds
-    const int pr = pr0 + (threadIdx.x & 255), qtr = threadIdx.x >> 8;
-    double s0 = 0.0, s1 = 0.0, rsn = 0.0, rcs = 1.0;
-    if (pr < npairs) {
-      const int h_lo = (p.H * qtr) / 4, h_hi = (p.H * (qtr + 1)) / 4;
-      for (int h0 = h_lo; h0 < h_hi; h0 += 16) {   // sixteen loads in flight, then the sums
-        float2 v[16];
+  const int h_lo = (p.H * g) / G, h_hi = (p.H * (g + 1)) / G;
+  const bool rotate = g == 0 && pr >= first_rope && ok;
+  double s0 = 0.0, s1 = 0.0, rsn = 0.0, rcs = 1.0;
+  bool have_angle = false;
+  for (int h0 = h_lo; h0 < h_hi; h0 += 16) {
+    float2 v[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          v[u] = h0 + u < h_hi ? __ldg(reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h0 + u) * p.D) + pr)
-                               : make_float2(0.f, 0.f);
-        if (h0 == h_lo && qtr == 0 && pr >= first_rope && ok)   // rotation angle while loads fly
-          sincos(static_cast<double>(L - 1) * rope_inv_freq(p, pr - first_rope), &rsn, &rcs);
+    for (int u = 0; u < 16; ++u)
+      v[u] = h0 + u < h_hi ? __ldg(reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h0 + u) * p.D) + pr)
+                           : make_float2(0.f, 0.f);
+    if (rotate && !have_angle) {  // rotation angle while the loads fly
+      sincos(static_cast<double>(L - 1) * rope_inv_freq(p, pr - first_rope), &rsn, &rcs);
+      have_angle = true;
+    }
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          s0 += v[u].x;
-          s1 += v[u].y;
-        }
-      }
+    for (int u = 0; u < 16; ++u) {
+      s0 += v[u].x;
+      s1 += v[u].y;
     }
-    part[qtr][0][threadIdx.x & 255] = s0;
-    part[qtr][1][threadIdx.x & 255] = s1;
-    __syncthreads();
-    if (qtr == 0 && pr < npairs) {
-      const int k = threadIdx.x & 255;
-      s0 = (part[0][0][k] + part[1][0][k]) + (part[2][0][k] + part[3][0][k]);
-      s1 = (part[0][1][k] + part[1][1][k]) + (part[2][1][k] + part[3][1][k]);
-      if (pr >= first_rope && ok) {
-        const double a = s0, c = s1;
-        s0 = a * rcs - c * rsn;
-        s1 = a * rsn + c * rcs;
-      }
-      reinterpret_cast<float2*>(ws.qbar + static_cast<int64_t>(b) * p.D)[pr] =
-          make_float2(static_cast<float>(s0 * scale), static_cast<float>(s1 * scale));
+  }
+  if (rotate && !have_angle)  // head group 0 holds no heads when H < G
+    sincos(static_cast<double>(L - 1) * rope_inv_freq(p, pr - first_rope), &rsn, &rcs);
+  part[tid][0] = s0;
+  part[tid][1] = s1;
+  __syncthreads();
+  if (g == 0) {
+    double a = 0.0, c = 0.0;
+    for (int gg = 0; gg < G; ++gg) {
+      a += part[gg * P + k][0];
+      c += part[gg * P + k][1];
     }
-    __syncthreads();
+    if (rotate) {
+      const double x = a;
+      a = x * rcs - c * rsn;
+      c = x * rsn + c * rcs;
+    }
+    const double scale = static_cast<double>(p.sm_scale) / p.H;
+    reinterpret_cast<float2*>(ws.qbar + static_cast<int64_t>(b) * p.D)[pr] =
+        make_float2(static_cast<float>(a * scale), static_cast<float>(c * scale));
   }
 }
 
@@ -544,92 +557,159 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, 
 }
 
 
-// Whole selection of one request in one CTA, for up to kSmallPerThread * 512 candidates: the
-// scores stay in registers (thread t holds a contiguous run of indices), three radix digits are
-// counted in shared memory, ties at the threshold key go to the lowest indices through a block
-// scan in index order, and the winners are written in ascending order by a second block scan.
+// Whole selection of one request in one CTA, for up to kSmallMax candidates. Thread t holds the
+// scores of the consecutive indices [t * per, (t + 1) * per) in registers, with per fixed by the
+// largest candidate count of the launch so that the loads are issued before the request's own
+// count has arrived. The three radix digits (11, 11, 10 bits of the order key) are resolved with
+// the histogram split across the block (thread t owns bins [t * NBL, (t + 1) * NBL)), two
+// barriers per digit; the first digit's histogram is the one the score kernel counted. Ties at
+// the threshold key go to the lowest indices and the winners are written in ascending order, both
+// from one block scan of the packed pair (count above the threshold, count equal to it).
 constexpr int kSmallThreads = 512;
+constexpr int kSmallWarps = kSmallThreads / 32;
 constexpr int kSmallPerThread = 32;
 constexpr int kSmallMax = kSmallThreads * kSmallPerThread;
 
+// Boundary of a block-distributed histogram for selecting `need` items from the top bin down:
+// returns (bin, items in the bins above it) to every thread.
+template <int NBL>
+__device__ __forceinline__ uint2 small_boundary(const uint32_t (&c)[NBL], uint32_t need, uint32_t* wsum,
+                                                uint2* bnd) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < NBL; ++i) s += c[i];
+  uint32_t suf = s;  // items in this lane's bins and those of the lanes above it
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += t;
+  }
+  if (lane == 0) wsum[w] = suf;
+  __syncthreads();
+  uint32_t above = (lane > w && lane < kSmallWarps) ? wsum[lane] : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+  above += suf - s;  // items in all bins above this thread's bins
+  if (above < need && above + s >= need) {
+    uint32_t cum = above;
+#pragma unroll
+    for (int i = NBL - 1; i >= 0; --i) {
+      if (cum + c[i] >= need) {
+        *bnd = make_uint2(static_cast<uint32_t>(threadIdx.x * NBL + i), cum);
+        break;
+      }
+      cum += c[i];
+    }
+  }
+  __syncthreads();
+  return *bnd;
+}
+
 __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* scores, int64_t stride,
-                                                                   int top_k, IndexerWs ws,
+                                                                   int nmax, int top_k, IndexerWs ws,
                                                                    int32_t* idx, int32_t* cnt) {
   griddep_wait();
   griddep_launch();
-  __shared__ uint32_t h[kHistBins];
-  __shared__ uint32_t sh[32];
-  __shared__ uint32_t bnd[2];
-  const int b = blockIdx.x;
-  const int N = ws.n_c[b];
-  const int k_eff = N < top_k ? N : top_k;
-  const int per = (N + kSmallThreads - 1) / kSmallThreads;
-  const int j0 = threadIdx.x * per;
-  int32_t* out = idx + static_cast<int64_t>(b) * top_k;
-  uint32_t key[kSmallPerThread];
+  __shared__ __align__(16) uint32_t h2[kHistBins];
+  __shared__ __align__(16) uint32_t h3[kHistBins / 2];
+  __shared__ uint32_t wsum[2][kSmallWarps];
+  __shared__ uint2 bnd;
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int per = (nmax + 4 * kSmallThreads - 1) / (4 * kSmallThreads) * 4;  // multiple of 4, <= 32
+  const int j0 = tid * per;
   const float* sb = scores + static_cast<int64_t>(b) * stride;
-#pragma unroll
-  for (int u = 0; u < kSmallPerThread; ++u) key[u] = (u < per && j0 + u < N) ? f32_order_key(__ldcg(sb + j0 + u)) : 0u;
 
-  uint32_t T = 0, idx_quota = 0;  // selected: key > T, or key == T among the first idx_quota
-  bool all = N <= top_k;
-  if (!all) {
-    uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k_eff);
+  // every load first: scores (16-byte vectors inside the padded row), first-digit histogram, count
+  float4 raw[kSmallPerThread / 4];
 #pragma unroll
-    for (int d = 0; d < 3; ++d) {
-      const int shift = d == 0 ? 21 : (d == 1 ? 10 : 0);
-      const int nb = d == 2 ? 1024 : 2048;
-      if (d == 0) {
-        // the first digit was counted by the score kernel
-        for (int i = threadIdx.x; i < nb; i += blockDim.x) h[i] = __ldcg(ws.hist + static_cast<int64_t>(b) * kHistBins + i);
-      } else {
-        for (int i = threadIdx.x; i < nb; i += blockDim.x) h[i] = 0;
-        __syncthreads();
+  for (int v = 0; v < kSmallPerThread / 4; ++v)
+    raw[v] = (4 * v < per && j0 + 4 * v < nmax) ? __ldcg(reinterpret_cast<const float4*>(sb + j0) + v)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  const uint4 c1v = __ldcg(reinterpret_cast<const uint4*>(ws.hist + static_cast<int64_t>(b) * kHistBins) + tid);
+  const int N = ws.n_c[b];
+  for (int i = tid; i < kHistBins; i += kSmallThreads) h2[i] = 0;
+  for (int i = tid; i < kHistBins / 2; i += kSmallThreads) h3[i] = 0;
+
+  uint32_t key[kSmallPerThread];
+  uint32_t valid = 0;
 #pragma unroll
-        for (int u = 0; u < kSmallPerThread; ++u)   // only keys in the boundary bin so far
-          if (u < per && j0 + u < N && (key[u] & mask) == prefix)
-            atomicAdd(h + ((key[u] >> shift) & (nb - 1)), 1u);
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) bnd[0] = bnd[1] = 0;
-      find_boundary(h, nb, need, true, sh, bnd);
-      need -= bnd[1];
-      prefix |= bnd[0] << shift;
-      mask |= static_cast<uint32_t>(nb - 1) << shift;
-      __syncthreads();
-    }
-    T = prefix;
-    idx_quota = need;   // how many of the key == T candidates are taken, lowest indices first
+  for (int v = 0; v < kSmallPerThread / 4; ++v) {
+    key[4 * v + 0] = f32_order_key(raw[v].x);
+    key[4 * v + 1] = f32_order_key(raw[v].y);
+    key[4 * v + 2] = f32_order_key(raw[v].z);
+    key[4 * v + 3] = f32_order_key(raw[v].w);
   }
-  // rank of each key == T among equals in index order
-  uint32_t n_eq = 0;
 #pragma unroll
   for (int u = 0; u < kSmallPerThread; ++u)
-    if (!all && u < per && j0 + u < N && key[u] == T) ++n_eq;
-  const uint32_t eq_incl = block_inclusive_scan<uint32_t>(n_eq, sh, nullptr);
-  uint32_t eq_rank = eq_incl - n_eq;
-  uint32_t sel_mask = 0, n_sel = 0;
+    if (u < per && j0 + u < N) valid |= 1u << u;
+
+  const int k_eff = N < top_k ? N : top_k;
+  const bool all = N <= top_k;
+  uint32_t T = 0, quota = 0;  // selected: key > T, and the first `quota` keys == T in index order
+  if (!all) {
+    const uint32_t c1[4] = {c1v.x, c1v.y, c1v.z, c1v.w};
+    const uint2 r1 = small_boundary<4>(c1, static_cast<uint32_t>(k_eff), wsum[0], &bnd);
+    const uint32_t need2 = static_cast<uint32_t>(k_eff) - r1.y;
+#pragma unroll
+    for (int u = 0; u < kSmallPerThread; ++u)
+      if (((valid >> u) & 1u) && (key[u] >> 21) == r1.x) atomicAdd(h2 + ((key[u] >> 10) & 2047u), 1u);
+    __syncthreads();
+    const uint4 c2v = reinterpret_cast<const uint4*>(h2)[tid];
+    const uint32_t c2[4] = {c2v.x, c2v.y, c2v.z, c2v.w};
+    const uint2 r2 = small_boundary<4>(c2, need2, wsum[1], &bnd);
+    const uint32_t need3 = need2 - r2.y;
+    const uint32_t p2 = (r1.x << 11) | r2.x;
+#pragma unroll
+    for (int u = 0; u < kSmallPerThread; ++u)
+      if (((valid >> u) & 1u) && (key[u] >> 10) == p2) atomicAdd(h3 + (key[u] & 1023u), 1u);
+    __syncthreads();
+    const uint2 c3v = reinterpret_cast<const uint2*>(h3)[tid];
+    const uint32_t c3[2] = {c3v.x, c3v.y};
+    const uint2 r3 = small_boundary<2>(c3, need3, wsum[0], &bnd);
+    T = (p2 << 10) | r3.x;
+    quota = need3 - r3.y;
+  }
+
+  // one exclusive block scan of (count above T) << 16 | (count equal to T), both <= kSmallMax
+  uint32_t n_gt = 0, n_eq = 0;
 #pragma unroll
   for (int u = 0; u < kSmallPerThread; ++u) {
-    if (u < per && j0 + u < N) {
+    if ((valid >> u) & 1u) {
+      n_gt += (all || key[u] > T) ? 1u : 0u;
+      n_eq += (!all && key[u] == T) ? 1u : 0u;
+    }
+  }
+  const uint32_t packed = (n_gt << 16) | n_eq;
+  const int lane = tid & 31, w = tid >> 5;
+  uint32_t incl = packed;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wsum[1][w] = incl;
+  __syncthreads();
+  uint32_t below = (lane < w) ? wsum[1][lane] : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+  const uint32_t excl = below + incl - packed;
+  uint32_t eq_before = excl & 0xffffu;
+  uint32_t pos = (excl >> 16) + (eq_before < quota ? eq_before : quota);
+  int32_t* out = idx + static_cast<int64_t>(b) * top_k;
+#pragma unroll
+  for (int u = 0; u < kSmallPerThread; ++u) {
+    if ((valid >> u) & 1u) {
       bool take = all || key[u] > T;
-      if (!all && key[u] == T) take = eq_rank++ < idx_quota;
+      if (!all && key[u] == T) take = eq_before++ < quota;
       if (take) {
-        sel_mask |= 1u << u;
-        ++n_sel;
+        if (pos < static_cast<uint32_t>(top_k)) out[pos] = j0 + u;
+        ++pos;
       }
     }
   }
-  const uint32_t sel_incl = block_inclusive_scan<uint32_t>(n_sel, sh, nullptr);
-  uint32_t pos = sel_incl - n_sel;
-#pragma unroll
-  for (int u = 0; u < kSmallPerThread; ++u)
-    if (sel_mask & (1u << u)) {
-      if (pos < static_cast<uint32_t>(top_k)) out[pos] = j0 + u;
-      ++pos;
-    }
-  for (int i = k_eff + threadIdx.x; i < top_k; i += blockDim.x) out[i] = -1;
-  if (threadIdx.x == 0) cnt[b] = k_eff;
+  for (int i = k_eff + tid; i < top_k; i += kSmallThreads) out[i] = -1;
+  if (tid == 0) cnt[b] = k_eff;
 }
 
 template <int DT, int NV, int U>
@@ -691,7 +771,7 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
                            cudaStream_t stream) {
   const int64_t stride = score_stride(p.r, max_seq_len);
   float* sc = scores ? scores : ws.scores;
-  cudaError_t e = launch_kernel(qbar_kernel, dim3(batch), dim3(kQbarThreads), 0, stream, p, seq_len,
+  cudaError_t e = launch_kernel(qbar_kernel, dim3(kQbarSlices, batch), dim3(kQbarThreads), 0, stream, p, seq_len,
                                 max_seq_len, q, ws, status);
   if (e != cudaSuccess) return e;
   switch (p.comp_dtype) {
@@ -704,7 +784,7 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
   const int64_t nmax = static_cast<int64_t>(max_seq_len) / p.r;
   if (nmax <= kSmallMax)   // every request's candidates fit one CTA's registers
     return launch_kernel(topk_small_kernel, dim3(batch), dim3(kSmallThreads), 0, stream,
-                         static_cast<const float*>(sc), stride, top_k, ws, idx, cnt);
+                         static_cast<const float*>(sc), stride, static_cast<int>(nmax), top_k, ws, idx, cnt);
   dim3 mgrid(static_cast<unsigned>(nmax > 0 ? (nmax + kMarkChunk - 1) / kMarkChunk : 1), batch);
   e = launch_kernel(topk_mark_kernel, mgrid, dim3(kThreads), 0, stream, static_cast<const float*>(sc),
                     stride, top_k, ws);
