@@ -284,12 +284,197 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------- one new token
+
+// Decode form: every request appends at most one token, so a call either writes one ring slot
+// (group unfinished) or folds one group (the token completes it), never both, and no group is
+// shared by two calls' ring reads and writes. The fold is split across CTAs by 64-dim slices
+// (blockIdx.x): slice s owns the rotary-aligned pairs [32 s, 32 s + 32) of the entry, the ring
+// and the window row, so r ring tokens are read by D/64 CTAs instead of one. Each slice rotates
+// the whole new token, because the window token's FP8 scale needs the amax of all its dims.
+constexpr int kSlicePairs = 32;
+constexpr int kRingPreload = 16;  // ring tokens per warp whose loads are issued at the start
+
+__global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArgs a) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ float w[256];
+  __shared__ float2 part[kAppendThreads / 32][kSlicePairs];
+  __shared__ float2 xs[kSlicePairs];
+  __shared__ float c[2 * kSlicePairs];
+  __shared__ float red[32];
+  const LayerParams& p = a.p;
+  const int b = blockIdx.y, slice = blockIdx.x, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, nw = kAppendThreads / 32;
+  const int npairs = p.D / 2;
+  const int sp = npairs < kSlicePairs ? npairs : kSlicePairs;
+  const int pr_lo = slice * sp;
+  const int64_t prev = a.prev_len[b];
+  int64_t row0 = b, n = 1;
+  if (a.cu_new) {
+    row0 = a.cu_new[b];
+    n = static_cast<int64_t>(a.cu_new[b + 1]) - row0;
+  }
+  if (n <= 0) return;
+  if (n != 1 || prev < 0 || prev + 1 > a.max_seq_len) {
+    if (tid == 0 && slice == 0) atomicOr(a.status, CKV_DEV_BAD_LENGTH);
+    return;
+  }
+  const int r = p.r;
+  const int64_t pos = prev, t0 = pos / r * r;
+  const bool complete = pos == t0 + r - 1;
+  const float* ring = p.res_kv + static_cast<int64_t>(b) * r * p.D;
+  float* ring_logit = p.res_logit + static_cast<int64_t>(b) * r;
+
+  // every load first: table rows, logits, the new token, this warp's first ring tokens
+  int64_t crow = -1;
+  const int n_ring = r - 1;  // ring tokens of a completed group: slots 0 .. r - 2
+  const int per = (n_ring + nw - 1) / nw;
+  const int tlo = warp * per, thi = min(n_ring, tlo + per);
+  float2 rx[kRingPreload];
+  if (complete) {
+    crow = comp_row(p, b, pos / r, a.status);
+    for (int t = tid; t < r; t += kAppendThreads) w[t] = t < r - 1 ? ring_logit[t] : a.logit_new[row0];
+#pragma unroll
+    for (int u = 0; u < kRingPreload; ++u) {
+      const int t = tlo + u;
+      rx[u] = (t < thi && lane < sp) ? reinterpret_cast<const float2*>(ring + static_cast<int64_t>(t) * p.D)[pr_lo + lane]
+                                     : make_float2(0.f, 0.f);
+    }
+  }
+  const int64_t wrow = p.W > 0 ? win_row(p, b, pos, a.status) : -1;
+  const float* raw = a.kv_new + row0 * p.D;
+  float2 x[kMaxPairsPerThread];
+  #pragma unroll
+  for (int k = 0; k < kMaxPairsPerThread; ++k) {
+    const int pr = tid + k * kAppendThreads;
+    x[k] = pr < npairs ? rotate_raw_pair(a, raw, pr, pos) : make_float2(0.f, 0.f);
+  }
+
+  // this slice's pairs of the rotated token: ring slot or fold input
+#pragma unroll
+  for (int k = 0; k < kMaxPairsPerThread; ++k) {
+    const int pr = tid + k * kAppendThreads;
+    if (pr < pr_lo || pr >= pr_lo + sp) continue;
+    if (complete) xs[pr - pr_lo] = x[k];
+    else reinterpret_cast<float2*>(p.res_kv + (static_cast<int64_t>(b) * r + pos % r) * p.D)[pr] = x[k];
+  }
+  if (!complete && slice == 0 && tid == 0) ring_logit[pos % r] = a.logit_new[row0];
+
+  // window row (the new token is always inside the window when W > 0)
+  if (p.W > 0) {
+    if (p.win_dtype == CKV_F32) {
+      if (wrow >= 0)
+#pragma unroll
+        for (int k = 0; k < kMaxPairsPerThread; ++k) {
+          const int pr = tid + k * kAppendThreads;
+          if (pr >= pr_lo && pr < pr_lo + sp) reinterpret_cast<float2*>(p.win_codes + wrow * p.win_row_bytes)[pr] = x[k];
+        }
+    } else {
+      float amax = 0.f;
+#pragma unroll
+      for (int k = 0; k < kMaxPairsPerThread; ++k)
+        amax = fmaxf(amax, fmaxf(fabsf(x[k].x), fabsf(x[k].y)));  // zero beyond npairs
+      amax = block_max(amax, red);
+      if (wrow >= 0) {
+        const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(p.win_codes + wrow * p.win_row_bytes);
+#pragma unroll
+        for (int k = 0; k < kMaxPairsPerThread; ++k) {
+          const int pr = tid + k * kAppendThreads;
+          if (pr < pr_lo || pr >= pr_lo + sp) continue;
+          const uint32_t c0 = f32_to_e4m3_satfinite(x[k].x / sc);
+          const uint32_t c1 = f32_to_e4m3_satfinite(x[k].y / sc);
+          dst[pr] = static_cast<uint16_t>(c0 | (c1 << 8));
+        }
+        if (slice == 0 && tid == 0) p.win_scales[wrow] = sc;
+      }
+    }
+  }
+  if (!complete) return;
+
+  // softmax weights of the group
+  __syncthreads();
+  if (warp == 0) {
+    float m = -INFINITY;
+    for (int t = lane; t < r; t += 32) m = fmaxf(m, w[t]);
+    m = warp_max(m);
+    float sum = 0.f;
+    for (int t = lane; t < r; t += 32) {
+      const float e = expf(w[t] - m);
+      w[t] = e;
+      sum += e;
+    }
+    sum = warp_sum(sum);
+    for (int t = lane; t < r; t += 32) w[t] = w[t] / sum;
+  }
+  __syncthreads();
+  // ring tokens: warp partial sums over its run of tokens, lane = pair of the slice
+  float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int u = 0; u < kRingPreload; ++u) {
+    const float wt = tlo + u < thi ? w[tlo + u] : 0.f;
+    acc.x = fmaf(wt, rx[u].x, acc.x);
+    acc.y = fmaf(wt, rx[u].y, acc.y);
+  }
+  for (int t = tlo + kRingPreload; t < thi; ++t) {  // r > 8 * kRingPreload + 1 only
+    const float2 v = lane < sp ? reinterpret_cast<const float2*>(ring + static_cast<int64_t>(t) * p.D)[pr_lo + lane]
+                               : make_float2(0.f, 0.f);
+    acc.x = fmaf(w[t], v.x, acc.x);
+    acc.y = fmaf(w[t], v.y, acc.y);
+  }
+  if (lane < sp) part[warp][lane] = acc;
+  __syncthreads();
+  if (tid < sp) {
+    float2 e = make_float2(0.f, 0.f);
+    for (int ww = 0; ww < nw; ++ww) {
+      e.x += part[ww][tid].x;
+      e.y += part[ww][tid].y;
+    }
+    e.x = fmaf(w[r - 1], xs[tid].x, e.x);
+    e.y = fmaf(w[r - 1], xs[tid].y, e.y);
+    c[2 * tid] = e.x;
+    c[2 * tid + 1] = e.y;
+  }
+  __syncthreads();
+  if (crow < 0) return;
+  // this slice's dims of the entry
+  const int d_lo = 2 * pr_lo, nd = 2 * sp;
+  uint8_t* dst = p.comp_codes + crow * p.comp_row_bytes;
+  if (p.comp_dtype == CKV_F32) {
+    if (tid < nd) reinterpret_cast<float*>(dst)[d_lo + tid] = c[tid];
+  } else if (p.comp_dtype == CKV_BF16) {
+    if (tid < nd) reinterpret_cast<uint16_t*>(dst)[d_lo + tid] = f32_to_bf16_rne(c[tid]);
+  } else if (tid < nd / 16) {  // NVFP4: one 16-element block per thread
+    const float* v = c + 16 * tid;
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+    const uint8_t sc = f32_to_e4m3_satfinite(amax / 6.0f);
+    const float s = e4m3_to_f32(sc);
+    uint32_t lo = 0, hi = 0;
+    if (s > 0.f) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lo |= static_cast<uint32_t>(f32_to_e2m1_satfinite(v[e] / s)) << (4 * e);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) hi |= static_cast<uint32_t>(f32_to_e2m1_satfinite(v[8 + e] / s)) << (4 * e);
+    }
+    const int blk = d_lo / 16 + tid;
+    reinterpret_cast<uint2*>(dst)[blk] = make_uint2(lo, hi);
+    p.comp_scales[crow * (p.D / 16) + blk] = sc;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_len,
                           const int32_t* cu_new, int max_new, int max_seq_len, const float* kv_new,
                           const float* logit_new, uint32_t* status, cudaStream_t stream) {
   AppendArgs a{p, prev_len, cu_new, max_seq_len, kv_new, logit_new, status};
+  if (max_new == 1) {  // one token per request: the fold split across 64-dim slices
+    const int slices = p.D / 2 < kSlicePairs ? 1 : p.D / 2 / kSlicePairs;
+    return launch_kernel(append_decode_kernel, dim3(slices, batch), dim3(kAppendThreads), 0, stream, a);
+  }
   const int64_t groups = static_cast<int64_t>(max_new) / p.r + 2;
   const int gx = static_cast<int>(groups < 512 ? groups : 512);
   dim3 grid(gx, batch);

@@ -21,6 +21,7 @@ namespace ckv {
 bool attention_tc_supported(const LayerParams& p);
 int attention_tc_tiles_per_split(int batch, int64_t max_keys);
 int attention_tc_tile_keys();
+int attention_tc_keys_per_split(int batch, int64_t max_keys);
 cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,
                                 int max_seq_len, const float* q, const int32_t* idx,
                                 const int32_t* cnt, int idx_stride, const AttnWs& ws,
@@ -344,7 +345,7 @@ AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_
   const int64_t sel = max_selected > 0 ? max_selected : static_cast<int64_t>(max_seq_len) / p.r;
   const int64_t keys = sel + (p.W < max_seq_len ? p.W : max_seq_len);
   w.keys_per_split = attention_tc_supported(p)
-                         ? attention_tc_tile_keys() * attention_tc_tiles_per_split(batch, keys)
+                         ? attention_tc_keys_per_split(batch, keys)
                          : kSimtKeys;
   w.splits = static_cast<int>(keys > 0 ? (keys + w.keys_per_split - 1) / w.keys_per_split : 1);
   const size_t n_slot = static_cast<size_t>(batch) * w.splits * p.H;

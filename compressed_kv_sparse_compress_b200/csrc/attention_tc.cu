@@ -299,8 +299,6 @@ template <int CT, int WT>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const float* q, const int32_t* idx,
     const int32_t* cnt, int idx_stride, AttnWs ws, uint32_t* status) {
-  griddep_wait();
-  griddep_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(base);
@@ -318,33 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
 
   const int b = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int L = seq_len[b];
-  if (L < 1 || L > max_seq_len) return;  // flagged by the combine
-  const int64_t n_c = L / p.r;
-  const int64_t n_sel = idx ? min(static_cast<int64_t>(max(cnt[b], 0)), static_cast<int64_t>(idx_stride)) : n_c;
-  const int64_t n_win = min(p.W, L);
-  const int64_t n_keys = n_sel + n_win;
-  const int64_t k_begin = static_cast<int64_t>(split) * ws.keys_per_split;
-  if (k_begin >= n_keys) return;
-  const int64_t k_end = min(n_keys, k_begin + ws.keys_per_split);
-  const int n_tiles = static_cast<int>((k_end - k_begin + kTile - 1) / kTile);
-
-  // ---- set-up: barriers; the prepared query image (64 KB, written per request by the prep
-  //      kernel) is bulk-copied into the Q region while the keys of tile 0 are resolved and staged
   const uint32_t bar_q = sb + kOffBarQ;
+
+  // ---- set-up that reads no global memory, before waiting for the previous kernel: barriers,
+  //      running max and sum, tensor memory
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(bar_q, 1);
     fence_proxy_async();
     flags[0] = flags[1] = 0;
-    const uint8_t* img = ws.qimage + static_cast<int64_t>(b) * kQBytes;
-    constexpr uint32_t kPiece = 16384;
-    mbar_expect_tx(bar_q, kQBytes);
-#pragma unroll 1
-    for (uint32_t off = 0; off < kQBytes; off += kPiece) bulk_g2s(sb + kOffQ + off, img + off, kPiece, bar_q);
   }
-  key_meta<WT>(p, b, L, idx, idx_stride, n_c, n_sel, n_win, k_begin, k_end, key_row, key_win, key_vs,
-               key_ls, status);
   if (tid < kH) {
     m_run[tid] = -INFINITY;
     l_run[tid] = 0.f;
@@ -354,25 +335,69 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  auto release = [&]() {   // every exit after the allocation (block-uniform)
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
+    }
+  };
+  griddep_wait();
+  griddep_launch();
+
+  const int L = seq_len[b];
+  if (L < 1 || L > max_seq_len) {  // flagged by the combine
+    release();
+    return;
+  }
+  const int64_t n_c = L / p.r;
+  const int64_t n_sel = idx ? min(static_cast<int64_t>(max(cnt[b], 0)), static_cast<int64_t>(idx_stride)) : n_c;
+  const int64_t n_win = min(p.W, L);
+  const int64_t n_keys = n_sel + n_win;
+  const int64_t k_begin = static_cast<int64_t>(split) * ws.keys_per_split;
+  if (k_begin >= n_keys) {
+    release();
+    return;
+  }
+  const int64_t k_end = min(n_keys, k_begin + ws.keys_per_split);
+  const int n_tiles = static_cast<int>((k_end - k_begin + kTile - 1) / kTile);
+
+  // ---- the prepared query image (64 KB, written per request by the prep kernel) is bulk-copied
+  //      into the Q region while the keys of tile 0 are resolved and staged
+  if (tid == 0) {
+    const uint8_t* img = ws.qimage + static_cast<int64_t>(b) * kQBytes;
+    constexpr uint32_t kPiece = 16384;
+    mbar_expect_tx(bar_q, kQBytes);
+#pragma unroll 1
+    for (uint32_t off = 0; off < kQBytes; off += kPiece) bulk_g2s(sb + kOffQ + off, img + off, kPiece, bar_q);
+  }
+  key_meta<WT>(p, b, L, idx, idx_stride, n_c, n_sel, n_win, k_begin, k_end, key_row, key_win, key_vs,
+               key_ls, status);
+  __syncthreads();
   uint32_t phase = 0;
   bool ok = true;
   bool q_ready = false;
 
   for (int tile = 0; tile < n_tiles && ok; ++tile) {
+    const int64_t k_first = k_begin + static_cast<int64_t>(tile) * kTile;
+    const int n_valid = static_cast<int>(min(static_cast<int64_t>(kTile), k_end - k_first));
     if (tile > 0) {
       key_meta<WT>(p, b, L, idx, idx_stride, n_c, n_sel, n_win, k_begin + static_cast<int64_t>(tile) * kTile,
                    k_end, key_row, key_win, key_vs, key_ls, status);
       __syncthreads();
     }
 
-    // ---- stage the tile as fp16 (absent keys are zero rows): warp w converts keys 16w .. 16w+15,
-    //      lane l the granules l and l + 32 of each (the key's row and kind read once per key)
+    // ---- stage the tile as fp16 (absent keys are zero rows): warp w converts keys 8w .. 8w+7 and,
+    //      when the tile holds more than 64 keys, 64+8w .. 64+8w+7; lane l the granules l and l+32
+    //      of each (the key's row and kind read once per key). Rows that are not staged hold
+    //      stale or uninitialised values: their logits are masked and no PV step reads them.
 #pragma unroll 1
-    for (int jb = 0; jb < 16; jb += 8) {
+    for (int jb = 0; jb < (n_valid > kTile / 2 ? 16 : 8); jb += 8) {
       Raw r[8][2];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int j = 16 * warp + jb + u;
+        const int j = 8 * jb + 8 * warp + u;
         const int64_t row = key_row[j];
         const bool win = key_win[j] != 0;
         r[u][0] = load_granule<CT, WT>(p, row, win, lane);
@@ -380,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int j = 16 * warp + jb + u;
+        const int j = 8 * jb + 8 * warp + u;
         const bool win = key_win[j] != 0;
         st_shared_v4(sb + kOffX + swz(kXChunk, j, lane), convert_granule<CT, WT>(r[u][0], win));
         st_shared_v4(sb + kOffX + swz(kXChunk, j, lane + 32), convert_granule<CT, WT>(r[u][1], win));
@@ -488,8 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     // ---- O^T += X^T . P^T
     if (tid == 128) {
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {   // consecutive MMAs go to different accumulators
+#pragma unroll 1
+      for (int kk = 0; kk < (n_valid + 15) / 16; ++kk) {   // consecutive MMAs go to different accumulators
         const uint64_t bp = sdesc(sb + kOffP + kk * 2048, 8192, 1024);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -523,12 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
     if (tid < kH) reinterpret_cast<float2*>(ws.part_ml)[slot + tid] = make_float2(-INFINITY, 0.f);
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
+  release();
 }
 
 template <int CT, int WT>
@@ -559,6 +579,14 @@ int attention_tc_tiles_per_split(int batch, int64_t max_keys) {
 }
 
 int attention_tc_tile_keys() { return kTile; }
+
+int attention_tc_keys_per_split(int batch, int64_t max_keys) {
+  // half tiles (64 keys; the MMAs still run at M = 128 over the staged half) while they fit one
+  // wave: twice the CTAs, each staging half the rows
+  const int64_t halves = static_cast<int64_t>(batch) * ((max_keys + kTile / 2 - 1) / (kTile / 2));
+  if (halves <= sm_count()) return kTile / 2;
+  return kTile * attention_tc_tiles_per_split(batch, max_keys);
+}
 
 cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,
                                 int max_seq_len, const float* q, const int32_t* idx,

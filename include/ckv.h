@@ -165,7 +165,9 @@ size_t ckv_attention_workspace_bytes(const ckv_layer_cfg* cfg, int32_t batch,
  *   d_prev_len  [batch] int32: tokens already appended (>= 0).
  *   d_cu_new    [batch+1] int32 prefix offsets into the rows of d_kv_new, or NULL for exactly one
  *               token per request (row b).
- *   max_new     host upper bound of n_b (1 when d_cu_new is NULL); sizes the grid.
+ *   max_new     host upper bound of n_b (1 when d_cu_new is NULL); sizes the grid. With
+ *               max_new == 1 (decode) a request with n_b > 1 is rejected on the device
+ *               (CKV_DEV_BAD_LENGTH, nothing written for it).
  *   max_seq_len host upper bound of prev_len[b] + n_b (table bounds).
  *   d_kv_new    [sum n_b][D] fp32;  d_logit_new [sum n_b] fp32.
  * The tables must map every logical block written: the blocks holding the completed entries
