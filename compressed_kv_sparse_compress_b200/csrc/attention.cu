@@ -15,6 +15,7 @@
 // combine. The tensor-core path for H=64 lives in attention_tc.cu and writes the same partials.
 
 #include "ckv_internal.h"
+#include "ckv_ptx.cuh"
 
 namespace ckv {
 
@@ -31,7 +32,6 @@ namespace {
 
 constexpr int kSimtThreads = 256;
 constexpr int kSimtKeys = 32;  // keys per split of the CUDA-core path
-constexpr int kCombineThreads = 128;
 
 struct KeyList {
   int64_t n_c, n_sel, n_win, n_keys;
@@ -231,97 +231,244 @@ __global__ void __launch_bounds__(kPrepThreads) attn_prep_kernel(LayerParams p, 
   }
 }
 
-__global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(
+// Merge of the splits of one (request, head) and inverse rotation for the CUDA-core path (fp32
+// partials), one thread per rotary-aligned pair of dims (D/2 threads). Every thread issues the
+// loads of its pair's partials for the first kCombineBatch splits before the split weights are
+// known; meanwhile the block reduces the splits' (m, l): M = max_s m_s, w_s = exp(m_s - M),
+// Z = sum_s w_s l_s (log-sum-exp merge).
+constexpr int kCombineBatch = 8;
+constexpr int kCombineSmemSplits = 1024;
+
+__global__ void __launch_bounds__(512, 3) attn_combine_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const int32_t* cnt, bool sparse,
     int idx_stride, AttnWs ws, float* out, uint32_t* status) {
   griddep_wait();
   griddep_launch();
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int D = p.D;
-  float* o = out + (static_cast<int64_t>(b) * p.H + h) * D;
+  __shared__ float wts[kCombineSmemSplits];
+  __shared__ float red[2][16];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int D = p.D, pr = tid;  // dims 2pr, 2pr + 1
+  float2* o = reinterpret_cast<float2*>(out + (static_cast<int64_t>(b) * p.H + h) * D);
   const int L = seq_len[b];
   if (L < 1 || L > max_seq_len) {
-    if (h == 0 && threadIdx.x == 0) atomicOr(status, CKV_DEV_BAD_LENGTH);
-    for (int d = threadIdx.x; d < D; d += blockDim.x) o[d] = 0.f;
+    if (h == 0 && tid == 0) atomicOr(status, CKV_DEV_BAD_LENGTH);
+    o[pr] = make_float2(0.f, 0.f);
     return;
+  }
+  const int first_rope = (D - p.d_r) / 2;
+  double rc = 1.0, rs = 0.0;  // rotation of this pair by the query position
+  if (pr >= first_rope) {
+    const double* rope = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
+    rc = rope[2 * (pr - first_rope)];
+    rs = rope[2 * (pr - first_rope) + 1];
   }
   const KeyList kl = key_list(p, L, cnt, sparse, idx_stride, b);
   const int ns = static_cast<int>((kl.n_keys + ws.keys_per_split - 1) / ws.keys_per_split);
-  // log-sum-exp merge of the splits: M = max of the split maxima, w_s = exp(m_s - M),
-  // Z = sum_s w_s l_s; the weights of the first kCombineSmemSplits splits are kept in shared memory
-  constexpr int kCombineSmemSplits = 256;
-  __shared__ float wts[kCombineSmemSplits];
-  __shared__ float red_m[32], red_z[32];
-  const float2* ml = reinterpret_cast<const float2*>(ws.part_ml);
   const int64_t base = static_cast<int64_t>(b) * ws.splits;
-  // one pass: each thread merges its splits' (m, l) online, then the block merges the threads
-  float mloc = -INFINITY, zloc = 0.f;
-  for (int s = threadIdx.x; s < ns; s += blockDim.x) {
-    const float2 v = __ldcg(ml + (base + s) * p.H + h);
-    if (s < kCombineSmemSplits) wts[s] = v.y > 0.f ? v.x : -INFINITY;
-    if (v.y > 0.f) {
-      const float mn = fmaxf(mloc, v.x);
-      zloc = zloc * expf(mloc - mn) + v.y * expf(v.x - mn);
-      mloc = mn;
-    }
+  const int64_t split_stride = static_cast<int64_t>(p.H) * D / 2;  // in pairs
+  const float2* po = reinterpret_cast<const float2*>(ws.part_o + (base * p.H + h) * D) + pr;
+  // this pair's partials of the first splits: in flight while the weights are reduced
+  float2 x[kCombineBatch];
+#pragma unroll
+  for (int u = 0; u < kCombineBatch; ++u) x[u] = u < ns ? __ldcg(po + u * split_stride) : make_float2(0.f, 0.f);
+
+  const float2* ml = reinterpret_cast<const float2*>(ws.part_ml);
+  float mloc = -INFINITY;
+  for (int sidx = tid; sidx < ns; sidx += blockDim.x) {
+    const float2 v = __ldcg(ml + (base + sidx) * p.H + h);
+    if (v.y > 0.f) mloc = fmaxf(mloc, v.x);  // l = 0: the split holds no keys (or gave up)
   }
-  const float mwarp = warp_max(mloc);
-  zloc = warp_sum(mloc == -INFINITY ? 0.f : zloc * expf(mloc - mwarp));
-  if ((threadIdx.x & 31) == 0) {
-    red_m[threadIdx.x >> 5] = mwarp;
-    red_z[threadIdx.x >> 5] = zloc;
-  }
+  mloc = warp_max(mloc);
+  if (lane == 0) red[0][warp] = mloc;
   __syncthreads();
   float M = -INFINITY;
-  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) M = fmaxf(M, red_m[i]);
-  float Z = 0.f;
-  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i)
-    if (red_m[i] > -INFINITY) Z += red_z[i] * expf(red_m[i] - M);
-  // split weights exp(m_s - M) for the first kCombineSmemSplits splits
-  for (int s = threadIdx.x; s < ns && s < kCombineSmemSplits; s += blockDim.x)
-    wts[s] = wts[s] > -INFINITY ? expf(wts[s] - M) : 0.f;
-  __syncthreads();
-  const float inv = Z > 0.f ? 1.f / Z : 0.f;
-  auto weight = [&](int s) -> float {
-    if (s < kCombineSmemSplits) return wts[s];
-    const float2 v = __ldcg(ml + (base + s) * p.H + h);
-    return v.y > 0.f ? expf(v.x - M) : 0.f;
-  };
-  const int first_rope = (D - p.d_r) / 2;
-  const double* rope = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
-  const float4* po = reinterpret_cast<const float4*>(ws.part_o + (base * p.H + h) * D);
-  const int64_t split_stride = static_cast<int64_t>(p.H) * D / 4;
-  for (int c = threadIdx.x; c < D / 4; c += blockDim.x) {   // dims 4c .. 4c+3 (two pairs)
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < ns; s0 += 8) {   // eight splits' loads in flight
-      float wgt[8];
-      float4 x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) wgt[u] = s0 + u < ns ? weight(s0 + u) : 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        x[u] = wgt[u] > 0.f ? __ldcg(po + (s0 + u) * split_stride + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        acc.x = fmaf(wgt[u], x[u].x, acc.x);
-        acc.y = fmaf(wgt[u], x[u].y, acc.y);
-        acc.z = fmaf(wgt[u], x[u].z, acc.z);
-        acc.w = fmaf(wgt[u], x[u].w, acc.w);
-      }
+  for (int i = 0; i < nw; ++i) M = fmaxf(M, red[0][i]);
+  float zloc = 0.f;
+  for (int sidx = tid; sidx < ns; sidx += blockDim.x) {
+    const float2 v = __ldcg(ml + (base + sidx) * p.H + h);
+    float wv = 0.f;
+    if (v.y > 0.f) {
+      wv = expf(v.x - M);
+      zloc = fmaf(wv, v.y, zloc);
     }
-    float v[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {   // inverse rotation by the query position
-      const int pr = 2 * c + k;
-      if (pr >= first_rope) {
-        const double cs = rope[2 * (pr - first_rope)], sn = rope[2 * (pr - first_rope) + 1];
-        const double a = v[2 * k], e = v[2 * k + 1];
-        v[2 * k] = static_cast<float>(a * cs + e * sn);
-        v[2 * k + 1] = static_cast<float>(e * cs - a * sn);
-      }
-    }
-    reinterpret_cast<float4*>(o)[c] = make_float4(v[0], v[1], v[2], v[3]);
+    if (sidx < kCombineSmemSplits) wts[sidx] = wv;
   }
+  zloc = warp_sum(zloc);
+  if (lane == 0) red[1][warp] = zloc;
+  __syncthreads();
+  float Z = 0.f;
+  for (int i = 0; i < nw; ++i) Z += red[1][i];
+  auto weight = [&](int sidx) -> float {
+    if (sidx < kCombineSmemSplits) return wts[sidx];
+    const float2 v = __ldcg(ml + (base + sidx) * p.H + h);
+    if (!(v.y > 0.f)) return 0.f;
+    return expf(v.x - M);
+  };
+  float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int u = 0; u < kCombineBatch; ++u) {
+    if (u < ns) {
+      const float wv = weight(u);
+      if (wv > 0.f) {
+        acc.x = fmaf(wv, x[u].x, acc.x);
+        acc.y = fmaf(wv, x[u].y, acc.y);
+      }
+    }
+  }
+  for (int s0 = kCombineBatch; s0 < ns; s0 += kCombineBatch) {
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u)
+      x[u] = s0 + u < ns ? __ldcg(po + (s0 + u) * split_stride) : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u) {
+      if (s0 + u < ns) {
+        const float wv = weight(s0 + u);
+        if (wv > 0.f) {
+          acc.x = fmaf(wv, x[u].x, acc.x);
+          acc.y = fmaf(wv, x[u].y, acc.y);
+        }
+      }
+    }
+  }
+  const float inv = Z > 0.f ? 1.f / Z : 0.f;
+  float vx = acc.x * inv, vy = acc.y * inv;
+  if (pr >= first_rope) {  // inverse rotation
+    const double a0 = vx, e0 = vy;
+    vx = static_cast<float>(a0 * rc + e0 * rs);
+    vy = static_cast<float>(e0 * rc - a0 * rs);
+  }
+  o[pr] = make_float2(vx, vy);
+}
+
+__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u) {
+  __half2_raw hr;
+  hr.x = static_cast<unsigned short>(u & 0xffffu);
+  hr.y = static_cast<unsigned short>(u >> 16);
+  return __half22float2(__half2(hr));
+}
+
+// Merge for the tensor-core path (H = 64, D = 512, fp16 partials O_s / c_s): one CTA per
+// (request, group of kGH heads). Each split's partial rows of the group are 4 KB of contiguous
+// memory; up to kGS splits per round are bulk-copied into shared memory while the block reduces
+// their (m, l) per head, and thread t then merges dims 8 (t % 64) .. 8 (t % 64) + 7 of head
+// t / 64 of the group from shared memory (running max and sums rescaled between rounds).
+constexpr int kGH = 4;
+constexpr int kGS = 16;
+constexpr int kGThreads = 256;
+constexpr int kGDim = 512;
+constexpr uint32_t kGRow = kGH * kGDim * 2;
+
+__global__ void __launch_bounds__(kGThreads, 1) attn_combine_tc_kernel(
+    LayerParams p, const int32_t* seq_len, int max_seq_len, const int32_t* cnt, bool sparse,
+    int idx_stride, int gs, AttnWs ws, float* out, uint32_t* status) {
+  griddep_wait();
+  griddep_launch();
+  extern __shared__ __align__(128) uint8_t cs_raw[];  // [gs][kGH][kGDim] fp16
+  __shared__ float wts[kGS][kGH];
+  __shared__ float red[2][kGThreads / 32];
+  __shared__ __align__(8) uint64_t bar_storage;
+  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int hh = tid >> 6, t64 = tid & 63;
+  const int h = g * kGH + hh;
+  float4* o = reinterpret_cast<float4*>(out + (static_cast<int64_t>(b) * p.H + h) * kGDim + 8 * t64);
+  const int L = seq_len[b];
+  if (L < 1 || L > max_seq_len) {
+    if (g == 0 && tid == 0) atomicOr(status, CKV_DEV_BAD_LENGTH);
+    o[0] = o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const uint32_t bar = smem_u32(&bar_storage);
+  if (tid == 0) mbar_init(bar, 1);
+  __syncthreads();
+  const KeyList kl = key_list(p, L, cnt, sparse, idx_stride, b);
+  const int ns = static_cast<int>((kl.n_keys + ws.keys_per_split - 1) / ws.keys_per_split);
+  const int64_t base = static_cast<int64_t>(b) * ws.splits;
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(ws.part_h + (base * p.H + g * kGH) * kGDim);
+  const int64_t split_bytes = static_cast<int64_t>(p.H) * kGDim * 2;
+  const float2* ml = reinterpret_cast<const float2*>(ws.part_ml);
+  float M = -INFINITY, Z = 0.f, acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  uint32_t phase = 0;
+  bool ok = true;
+  for (int s0 = 0; s0 < ns && ok; s0 += gs) {
+    const int nb = min(gs, ns - s0);
+    if (tid == 0) {
+      fence_proxy_async();  // earlier rounds' reads of the buffer come before the copies
+      mbar_expect_tx(bar, static_cast<uint32_t>(nb) * kGRow);
+      for (int u = 0; u < nb; ++u)
+        bulk_g2s(smem_u32(cs_raw + u * kGRow), src + (s0 + u) * split_bytes, kGRow, bar);
+    }
+    // weights of this round's splits, per head (64 threads per head: 2 warps)
+    float2 v = make_float2(-INFINITY, 0.f);
+    float scv = 0.f;
+    if (t64 < nb) {
+      v = __ldcg(ml + (base + s0 + t64) * p.H + h);
+      scv = __ldcg(ws.part_sc + (base + s0 + t64) * p.H + h);
+    }
+    const bool live = t64 < nb && v.y > 0.f;  // l = 0: the split holds no keys (or gave up)
+    const float mw = warp_max(live ? v.x : -INFINITY);
+    if (lane == 0) red[0][warp] = mw;
+    __syncthreads();
+    const float Mn = fmaxf(M, fmaxf(red[0][2 * hh], red[0][2 * hh + 1]));
+    float w = 0.f, zl = 0.f;
+    if (live) {
+      w = expf(v.x - Mn);
+      zl = w * v.y;
+      w *= scv;
+    }
+    if (t64 < nb) wts[t64][hh] = w;
+    zl = warp_sum(zl);
+    if (lane == 0) red[1][warp] = zl;
+    __syncthreads();
+    const float f = M == -INFINITY ? 0.f : expf(M - Mn);
+    Z = Z * f + (red[1][2 * hh] + red[1][2 * hh + 1]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] *= f;
+    M = Mn;
+    ok = __syncthreads_and(mbar_wait(bar, phase)) != 0;
+    phase ^= 1;
+    if (!ok) break;
+    for (int u = 0; u < nb; ++u) {
+      const float wu = wts[u][hh];
+      if (wu > 0.f) {
+        const uint4 r = *reinterpret_cast<const uint4*>(cs_raw + u * kGRow + hh * (kGDim * 2) + 16 * t64);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 x = half2_bits_to_float2(k == 0 ? r.x : k == 1 ? r.y : k == 2 ? r.z : r.w);
+          acc[2 * k] = fmaf(wu, x.x, acc[2 * k]);
+          acc[2 * k + 1] = fmaf(wu, x.y, acc[2 * k + 1]);
+        }
+      }
+    }
+    __syncthreads();  // the buffer, weights and reductions are reused by the next round
+  }
+  if (!ok) {
+    if (tid == 0) atomicOr(status, CKV_DEV_TIMEOUT);
+    mbar_wait(bar, phase ^ 1);  // let this round's copies land before the CTA exits (bounded)
+    o[0] = o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const float inv = Z > 0.f ? 1.f / Z : 0.f;
+  float v8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v8[k] = acc[k] * inv;
+  const int first_rope = (kGDim - p.d_r) / 2;
+  const double* rope = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {  // inverse rotation by the query position
+    const int pr = 4 * t64 + k;
+    if (pr >= first_rope) {
+      const double cs = rope[2 * (pr - first_rope)], sn = rope[2 * (pr - first_rope) + 1];
+      const double a0 = v8[2 * k], e0 = v8[2 * k + 1];
+      v8[2 * k] = static_cast<float>(a0 * cs + e0 * sn);
+      v8[2 * k + 1] = static_cast<float>(e0 * cs - a0 * sn);
+    }
+  }
+  o[0] = make_float4(v8[0], v8[1], v8[2], v8[3]);
+  o[1] = make_float4(v8[4], v8[5], v8[6], v8[7]);
 }
 
 template <int D>
@@ -351,16 +498,20 @@ AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_
   const size_t n_slot = static_cast<size_t>(batch) * w.splits * p.H;
   const size_t o_bytes = align_up(n_slot * p.D * sizeof(float), 256);
   const size_t ml_bytes = align_up(n_slot * 2 * sizeof(float), 256);
+  const size_t sc_bytes = align_up(n_slot * sizeof(float), 256);
   const size_t rope_bytes = align_up(static_cast<size_t>(batch) * (p.d_r / 2 + 1) * 2 * sizeof(double), 256);
   const size_t q_bytes = attention_tc_supported(p) ? static_cast<size_t>(batch) * kQImageBytes : 0;
+  w.half_parts = attention_tc_supported(p);
   if (base) {
     char* c = static_cast<char*>(base);
     w.part_o = reinterpret_cast<float*>(c);
+    w.part_h = reinterpret_cast<uint16_t*>(c);
     w.part_ml = reinterpret_cast<float*>(c + o_bytes);
     w.rope = reinterpret_cast<double*>(c + o_bytes + ml_bytes);
     w.qimage = q_bytes ? reinterpret_cast<uint8_t*>(c + o_bytes + ml_bytes + rope_bytes) : nullptr;
+    w.part_sc = reinterpret_cast<float*>(c + o_bytes + ml_bytes + rope_bytes + q_bytes);
   }
-  w.bytes = o_bytes + ml_bytes + rope_bytes + q_bytes;
+  w.bytes = o_bytes + ml_bytes + rope_bytes + q_bytes + sc_bytes;
   return w;
 }
 
@@ -388,8 +539,17 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
   prof_end(kProfAttention, stream);
   if (e != cudaSuccess) return e;
   dim3 grid(p.H, batch);
-  return launch_kernel(attn_combine_kernel, grid, dim3(kCombineThreads), 0, stream, p, seq_len,
-                       max_seq_len, cnt, idx != nullptr, idx_stride, ws, out, status);
+  if (ws.half_parts) {   // tensor-core path: H = 64, D = 512
+    const int gs = ws.splits < kGS ? ws.splits : kGS;
+    const int smem = gs * static_cast<int>(kGRow);
+    e = allow_smem(reinterpret_cast<const void*>(attn_combine_tc_kernel), smem);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(attn_combine_tc_kernel, dim3(p.H / kGH, batch), dim3(kGThreads), smem, stream, p,
+                         seq_len, max_seq_len, cnt, idx != nullptr, idx_stride, gs, ws, out, status);
+  }
+  const dim3 block(p.D / 2);   // one thread per pair of dims: 32 .. 512
+  return launch_kernel(attn_combine_kernel, grid, block, 0, stream, p, seq_len, max_seq_len, cnt,
+                       idx != nullptr, idx_stride, ws, out, status);
 }
 
 }  // namespace ckv

@@ -15,8 +15,9 @@
 // converted to fp16 while it is staged: bf16 and e2m1 x e4m3 values are exact in fp16 (|x| <
 // 65504), FP8 window codes are exact and their per-token scale is applied to the logits and to
 // P in fp32. Q~ (rotated query) is rounded to fp16 once. S^T (64 columns) and O^T (4 blocks of 64
-// columns) live in tensor memory. Each thread of warps 0-3 owns one key (one TMEM lane) for the
-// softmax; per-head maxima and sums are reduced across the 128 keys of a tile with warp
+// columns) live in tensor memory. The CTA has 32 warps, so that the gather of a tile's key rows
+// has many loads in flight; for the softmax warp w owns the keys of TMEM lane quarter w%4 (one
+// key per thread) and 8 heads; per-head maxima and sums are reduced across the keys with warp
 // reduce-scatters. The running maximum is only raised when a tile's maximum exceeds it by more
 // than 8 (then O^T is rescaled in tensor memory), so P <= e^8 stays well inside fp16.
 //
@@ -33,7 +34,7 @@ namespace {
 constexpr int kH = 64;
 constexpr int kD = 512;
 constexpr int kTile = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 1024;  // 32 warps: many loads in flight per SM while staging
 constexpr int kChunks = kD / 64;
 constexpr uint32_t kXChunk = kTile * 128;        // bytes of one 64-element chunk of the tile
 constexpr uint32_t kXBytes = kXChunk * kChunks;  // 128 KB
@@ -123,30 +124,16 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 constexpr uint32_t kIdescS = (1u << 4) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = kIdescS | (1u << 15) | (1u << 16);  // A and B MN-major
 
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};\n"
-               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
-               : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-               : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n"
-               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n"
+               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -181,6 +168,20 @@ __device__ __forceinline__ void reduce_scatter(float (&t)[N], int lane) {
       t[i] = kMax ? fmaxf(keep, recv) : keep + recv;
     }
   }
+}
+
+// Reduction of one value per (head of 8, lane) over the warp's 32 lanes: three reduce-scatter
+// stages, then two butterfly stages; lane l returns the reduction of entry l >> 2.
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce8(float (&t)[8], int lane) {
+  reduce_scatter<8, kMax>(t, lane);
+  float v = t[0];
+#pragma unroll
+  for (int o = 2; o > 0; o >>= 1) {
+    const float x = __shfl_xor_sync(0xffffffffu, v, o);
+    v = kMax ? fmaxf(v, x) : v + x;
+  }
+  return v;
 }
 
 // raw bytes of one 8-element granule of a key, loaded before conversion
@@ -388,27 +389,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       __syncthreads();
     }
 
-    // ---- stage the tile as fp16 (absent keys are zero rows): warp w converts keys 8w .. 8w+7 and,
-    //      when the tile holds more than 64 keys, 64+8w .. 64+8w+7; lane l the granules l and l+32
-    //      of each (the key's row and kind read once per key). Rows that are not staged hold
-    //      stale or uninitialised values: their logits are masked and no PV step reads them.
-#pragma unroll 1
-    for (int jb = 0; jb < (n_valid > kTile / 2 ? 16 : 8); jb += 8) {
-      Raw r[8][2];
+    // ---- stage the tile as fp16 (absent keys are zero rows): warp w converts kpw consecutive
+    //      keys (4 of a full tile, 2 when it holds at most 64 keys), lane l the granules l and l+32
+    //      of each (the key's row and kind read once per key), all of them in flight at once. Rows
+    //      that are not staged hold stale or uninitialised values: their logits are masked and no
+    //      PV step reads them.
+    {
+      constexpr int kB = (CT == CKV_F32 || WT == CKV_F32) ? 2 : 4;  // fp32 granules are 32 bytes
+      const int kpw = n_valid > kTile / 2 ? 4 : 2;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = 8 * jb + 8 * warp + u;
-        const int64_t row = key_row[j];
-        const bool win = key_win[j] != 0;
-        r[u][0] = load_granule<CT, WT>(p, row, win, lane);
-        r[u][1] = load_granule<CT, WT>(p, row, win, lane + 32);
-      }
+      for (int u0 = 0; u0 < 4; u0 += kB) {
+        if (u0 >= kpw) break;
+        Raw r[kB][2];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = 8 * jb + 8 * warp + u;
-        const bool win = key_win[j] != 0;
-        st_shared_v4(sb + kOffX + swz(kXChunk, j, lane), convert_granule<CT, WT>(r[u][0], win));
-        st_shared_v4(sb + kOffX + swz(kXChunk, j, lane + 32), convert_granule<CT, WT>(r[u][1], win));
+        for (int u = 0; u < kB; ++u) {
+          if (u0 + u < kpw) {
+            const int j = kpw * warp + u0 + u;
+            const int64_t row = key_row[j];
+            const bool win = key_win[j] != 0;
+            r[u][0] = load_granule<CT, WT>(p, row, win, lane);
+            r[u][1] = load_granule<CT, WT>(p, row, win, lane + 32);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          if (u0 + u < kpw) {
+            const int j = kpw * warp + u0 + u;
+            const bool win = key_win[j] != 0;
+            st_shared_v4(sb + kOffX + swz(kXChunk, j, lane), convert_granule<CT, WT>(r[u][0], win));
+            st_shared_v4(sb + kOffX + swz(kXChunk, j, lane + 32), convert_granule<CT, WT>(r[u][1], win));
+          }
+        }
       }
     }
     fence_proxy_async();
@@ -440,23 +451,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     if (!ok) break;
 
     // ---- softmax over the tile's keys: key j = TMEM lane; warp w reads the lanes of quarter w%4
-    //      and the 32 heads of half w/4
+    //      and the 8 heads of group w/4
     {
-      const int q4 = warp & 3, half = warp >> 2;
+      const int q4 = warp & 3, hg = warp >> 2;
       const int j = q4 * 32 + lane;
       const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-      uint32_t raw[32];
-      tmem_ld32(tmem + lane_base + kSCol + 32 * half, raw);
+      uint32_t raw[8];
+      tmem_ld8(tmem + lane_base + kSCol + 8 * hg, raw);
       const float f = key_ls[j];
       const bool valid = key_row[j] >= 0;
-      float sv[32], t[32];
+      float sv[8], t[8];
 #pragma unroll
-      for (int h = 0; h < 32; ++h) {
+      for (int h = 0; h < 8; ++h) {
         sv[h] = valid ? __uint_as_float(raw[h]) * f : -INFINITY;
         t[h] = sv[h];
       }
-      reduce_scatter<32, true>(t, lane);
-      red[q4 * kH + 32 * half + lane] = t[0];
+      const float mx = warp_reduce8<true>(t, lane);
+      if ((lane & 3) == 0) red[q4 * kH + 8 * hg + (lane >> 2)] = mx;
       __syncthreads();
       if (tid < kH) {
         const float mt = fmaxf(fmaxf(red[tid], red[kH + tid]), fmaxf(red[2 * kH + tid], red[3 * kH + tid]));
@@ -472,23 +483,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       }
       __syncthreads();
       const float vs = key_vs[j];
-      uint32_t packed[16];
+      uint32_t packed[4];
 #pragma unroll
-      for (int h = 0; h < 32; h += 2) {
-        const float m0 = m_run[32 * half + h], m1 = m_run[32 * half + h + 1];
+      for (int h = 0; h < 8; h += 2) {
+        const float m0 = m_run[8 * hg + h], m1 = m_run[8 * hg + h + 1];
         const float p0 = m0 == -INFINITY ? 0.f : __expf(sv[h] - m0);
         const float p1 = m1 == -INFINITY ? 0.f : __expf(sv[h + 1] - m1);
         t[h] = p0;
         t[h + 1] = p1;
         packed[h >> 1] = pack_f32x2(p0 * vs, p1 * vs);
       }
-#pragma unroll
-      for (int g = 0; g < 4; ++g)
-        st_shared_v4(sb + kOffP + static_cast<uint32_t>(j) * 128u +
-                         (static_cast<uint32_t>((4 * half + g) ^ (j & 7)) << 4),
-                     make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]));
-      reduce_scatter<32, false>(t, lane);
-      red[q4 * kH + 32 * half + lane] = t[0];
+      st_shared_v4(sb + kOffP + static_cast<uint32_t>(j) * 128u + (static_cast<uint32_t>(hg ^ (j & 7)) << 4),
+                   make_uint4(packed[0], packed[1], packed[2], packed[3]));
+      const float sm = warp_reduce8<false>(t, lane);
+      if ((lane & 3) == 0) red[q4 * kH + 8 * hg + (lane >> 2)] = sm;
       __syncthreads();
       if (tid < kH)
         l_run[tid] = l_run[tid] * alpha[tid] + ((red[tid] + red[kH + tid]) + (red[2 * kH + tid] + red[3 * kH + tid]));
@@ -496,12 +504,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       if (tile > 0 && flags[0]) {
 #pragma unroll 1
         for (int m = 0; m < 4; ++m) {
-          const uint32_t ta = tmem + lane_base + kOCol + 64 * m + 32 * half;
-          uint32_t o[32];
-          tmem_ld32(ta, o);
+          const uint32_t ta = tmem + lane_base + kOCol + 64 * m + 8 * hg;
+          uint32_t o[8];
+          tmem_ld8(ta, o);
 #pragma unroll
-          for (int h = 0; h < 32; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[32 * half + h]);
-          tmem_st32(ta, o);
+          for (int h = 0; h < 8; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[8 * hg + h]);
+          tmem_st8(ta, o);
         }
       }
       fence_proxy_async();
@@ -529,17 +537,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     tc_fence_after();
   }
 
-  // ---- partial outputs: O^T lane = dim, column = head (warp w: lane quarter w%4, heads of half w/4)
+  // ---- partial outputs: O^T lane = dim, column = head (warp w: lane quarter w%4, heads of
+  //      group w/4). Each head's row is stored as fp16 after division by a power of two 2^e,
+  //      e = (exponent of the row's max |o|) - 15 (at least -126), so that every value lies below
+  //      2^15 in magnitude with a relative step of 2^-11 of the row's max; e goes to part_sc.
   if (ok) {
-    const int q4 = warp & 3, half = warp >> 2;
+    const int q4 = warp & 3, hg = warp >> 2;
     const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
-#pragma unroll 1
-    for (int m = 0; m < 4; ++m) {
-      uint32_t o[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + kOCol + 64 * m + 32 * half, o);
-      const int d = 128 * m + 32 * q4 + lane;
+    uint32_t o[4][8];
 #pragma unroll
-      for (int h = 0; h < 32; ++h) ws.part_o[(slot + 32 * half + h) * kD + d] = __uint_as_float(o[h]);
+    for (int m = 0; m < 4; ++m)
+      tmem_ld8(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + kOCol + 64 * m + 8 * hg, o[m]);
+    float t[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+      t[h] = fmaxf(fmaxf(fabsf(__uint_as_float(o[0][h])), fabsf(__uint_as_float(o[1][h]))),
+                   fmaxf(fabsf(__uint_as_float(o[2][h])), fabsf(__uint_as_float(o[3][h]))));
+    const float amax_w = warp_reduce8<true>(t, lane);
+    if ((lane & 3) == 0) red[q4 * kH + 8 * hg + (lane >> 2)] = amax_w;
+    __syncthreads();
+    if (tid < kH) {
+      const float amax = fmaxf(fmaxf(red[tid], red[kH + tid]), fmaxf(red[2 * kH + tid], red[3 * kH + tid]));
+      int ex = 0;
+      float sc = 1.f;
+      if (amax > 0.f && amax <= 3.4e38f) {   // finite, non-zero
+        frexpf(amax, &ex);                    // amax = f * 2^ex, f in [0.5, 1)
+        sc = ldexpf(1.f, ex - 15 > -126 ? ex - 15 : -126);
+      }
+      alpha[tid] = sc;
+      ws.part_sc[slot + tid] = sc;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const float inv = 1.f / alpha[8 * hg + h];   // exact: a power of two
+      __half* dst = reinterpret_cast<__half*>(ws.part_h) + (slot + 8 * hg + h) * kD + 32 * q4 + lane;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) dst[128 * m] = __float2half_rn(__uint_as_float(o[m][h]) * inv);
     }
     if (tid < kH) reinterpret_cast<float2*>(ws.part_ml)[slot + tid] = make_float2(m_run[tid], l_run[tid]);
   }

@@ -71,7 +71,11 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
 
 // ---------------------------------------------------------------------------- attention
 struct AttnWs {
-  float* part_o;     // [B][S][H][D]   un-normalised partial outputs
+  float* part_o;     // [B][S][H][D]   un-normalised partial outputs (CUDA-core path)
+  uint16_t* part_h;  // [B][S][H][D]   tensor-core path: fp16 partial outputs divided by part_sc
+                     //                (same memory as part_o)
+  float* part_sc;    // [B][S][H]      tensor-core path: power-of-two scale of each partial
+  bool half_parts;   // which of the two forms the splits write
   float* part_ml;    // [B][S][H][2]   running max and sum of each split
   double* rope;      // [B][d_r/2][2]  cos, sin of each rotary pair at the query position
   uint8_t* qimage;   // [B][H*D*2]     tensor-core path: rotated fp16 query in the swizzled
