@@ -258,15 +258,38 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int b
   constexpr int EPV = VecFmt<DT>::kElems;
   static_assert(U <= LPE, "one writer lane per entry of a pass");
 
-  extern __shared__ int32_t chunk_prefix[];  // [batch + 1]
+  extern __shared__ int32_t chunk_prefix[];  // [batch + 1], then the candidate counts [batch]
+  int32_t* n_c = chunk_prefix + batch + 1;
   __shared__ int32_t scan_sh[32];
-  // chunks per request, exclusive prefix over the batch
-  {
+  // chunks per request, exclusive prefix over the batch (one warp when the batch fits it)
+  if (batch <= 32) {
+    if (threadIdx.x < 32) {
+      const int bb = threadIdx.x;
+      const int32_t n = bb < batch ? ws.n_c[bb] : 0;
+      const int32_t s = (n + CH - 1) / CH;
+      int32_t incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (bb >= o) incl += t;
+      }
+      if (bb < batch) {
+        n_c[bb] = n;
+        chunk_prefix[bb] = incl - s;
+      }
+      if (bb == 31) chunk_prefix[batch] = incl;
+    }
+    __syncthreads();
+  } else {
     const int per = (batch + blockDim.x - 1) / blockDim.x;
     int32_t s = 0;
     for (int i = 0; i < per; ++i) {
       const int bb = threadIdx.x * per + i;
-      if (bb < batch) s += (ws.n_c[bb] + CH - 1) / CH;
+      if (bb < batch) {
+        const int32_t n = ws.n_c[bb];
+        n_c[bb] = n;
+        s += (n + CH - 1) / CH;
+      }
     }
     int32_t total;
     const int32_t incl = block_inclusive_scan<int32_t>(s, scan_sh, &total);
@@ -275,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int b
       const int bb = threadIdx.x * per + i;
       if (bb < batch) {
         chunk_prefix[bb] = run;
-        run += (ws.n_c[bb] + CH - 1) / CH;
+        run += (n_c[bb] + CH - 1) / CH;
       }
     }
     if (threadIdx.x == 0) chunk_prefix[batch] = total;
@@ -304,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int b
       if (chunk_prefix[mid] <= ch) lo = mid; else hi = mid;
     }
     c.b = lo;
-    c.N = ws.n_c[lo];
+    c.N = n_c[lo];
     c.e_base = (ch - chunk_prefix[lo]) * CH;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -719,7 +742,7 @@ cudaError_t launch_score(const LayerParams& p, int batch, int max_seq_len, const
   constexpr int CH = U * (32 / LPE);
   const int64_t per_req = (static_cast<int64_t>(max_seq_len) / p.r + CH - 1) / CH;
   const int64_t chunks = per_req * batch;
-  const int smem = static_cast<int>(sizeof(int32_t) * (batch + 1));
+  const int smem = static_cast<int>(sizeof(int32_t) * (2 * batch + 1));
   auto kern = score_kernel<DT, NV, U>;
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
