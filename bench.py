@@ -178,8 +178,8 @@ def traffic_record(kernel: str, workload: str):
 class Step:
     """All layers of a workload on one GPU, with the step's inputs resident in HBM."""
 
-    def __init__(self, ckv, w: S.Workload, seed_offset: int = 0):
-        self.ckv, self.w = ckv, w
+    def __init__(self, ckv, w: S.Workload, seed_offset: int = 0, api: str = "fused"):
+        self.ckv, self.w, self.api = ckv, w, api
         wseed = S.Workload(w.name, w.seq_lens, w.num_heads, w.head_dim, w.rope_dim, w.window,
                            w.layers, w.paged, w.from_scratch, w.seed + seed_offset, w.description)
         self.gen = S.generate(wseed, "cuda")
@@ -209,7 +209,10 @@ class Step:
             q = lay["q"] if q_list is None else q_list[i]
             kv = lay["kv_new"] if kv_list is None else kv_list[i]
             lg = lay["logit_new"] if lg_list is None else lg_list[i]
-            outs.append(dl.step(seq, prev, q, kv, lg))
+            if self.api == "fused":
+                outs.append(dl.fused_step(seq, q, kv, lg))
+            else:
+                outs.append(dl.step(seq, prev, q, kv, lg))
         return outs
 
     def status(self) -> int:
@@ -226,7 +229,7 @@ def run_cuda(args, w: S.Workload):
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
-    step = Step(ckv, w, seed_offset=rank)
+    step = Step(ckv, w, seed_offset=rank, api=args.api)
     flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_sink = torch.empty(1, dtype=torch.float32, device=dev)
@@ -296,7 +299,10 @@ def run_cuda(args, w: S.Workload):
                     k += 1
                 else:
                     ckv.profile_events(prof_which)
-                dl.step(step.seq, step.prev, lay["q"], lay["kv_new"], lay["logit_new"])
+                if args.api == "fused":
+                    dl.fused_step(step.seq, lay["q"], lay["kv_new"], lay["logit_new"])
+                else:
+                    dl.step(step.seq, step.prev, lay["q"], lay["kv_new"], lay["logit_new"])
         kstep[i][1].record(stream)
     barrier()
     ckv.profile_events(prof_which)
@@ -367,6 +373,8 @@ def run_cuda(args, w: S.Workload):
             "l2": "flushed before every step outside the step events: 256 MiB written, then another "
                   "256 MiB read (the written lines are evicted before the step)",
             "step": "append decode token + indexer/top-k + attention (+ split combine), per layer",
+            "api": ("ckv_decode_step, one call per layer" if args.api == "fused"
+                    else "kv_compress_append + sparse_indexer_topk + compressed_window_attention"),
         },
         "hbm": {"step_bytes": step_bytes,
                 "step_GBps": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
@@ -501,6 +509,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(S.WORKLOADS))
     ap.add_argument("--impl", default="ckv", choices=["ckv", "reference"])
+    ap.add_argument("--api", default="fused", choices=["fused", "calls"],
+                    help="fused: one ckv_decode_step per layer; calls: append, select, attend")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-requests", type=int, default=0,

@@ -37,7 +37,8 @@ EXPORTS = (
     "kv_block_pool_num_free", "ckv_cache_row_bytes", "ckv_score_stride",
     "ckv_indexer_workspace_bytes", "ckv_attention_workspace_bytes", "kv_compress_append",
     "sparse_indexer_topk", "compressed_window_attention", "ckv_status_str", "ckv_launch_count",
-    "ckv_profile_events", "sparse_indexer_topk_noalloc",
+    "ckv_profile_events", "sparse_indexer_topk_noalloc", "ckv_decode_step_workspace_bytes",
+    "ckv_decode_step",
 )
 CKV_PROF_SCORE, CKV_PROF_ATTENTION = 0, 1
 
@@ -101,6 +102,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_indexer_topk_noalloc.argtypes = [P(LayerCfgC), P(LayerCacheC), i32, vp, i32, vp, i32,
                                                 vp, vp, vp, vp, vp]
     lib.sparse_indexer_topk_noalloc.restype = ctypes.c_int
+    lib.ckv_decode_step_workspace_bytes.argtypes = [P(LayerCfgC), i32, i32, i32]
+    lib.ckv_decode_step_workspace_bytes.restype = sz
+    lib.ckv_decode_step.argtypes = [P(LayerCfgC), P(LayerCacheC), i32, vp, i32, vp, vp, vp, i32, vp,
+                                    vp, vp, vp, sz, vp, vp]
+    lib.ckv_decode_step.restype = ctypes.c_int
     lib.ckv_status_str.argtypes = [ctypes.c_int]
     lib.ckv_status_str.restype = ctypes.c_char_p
     lib.ckv_profile_events.argtypes = [ctypes.c_int, vp, vp]
@@ -302,3 +308,20 @@ def compressed_window_attention(cfg: LayerConfig, cache: LayerCache, seq_len: to
         ctypes.byref(cfg.c()), ctypes.byref(cache.c()), batch, _ptr(seq_len), max_seq_len,
         _ptr(q), _ptr(idx), _ptr(cnt), stride, _ptr(out), _ptr(workspace), workspace.numel(),
         _ptr(status), _stream(stream)))
+
+
+def decode_step_workspace_bytes(cfg: LayerConfig, batch: int, max_seq_len: int, top_k: int) -> int:
+    return int(load_library().ckv_decode_step_workspace_bytes(ctypes.byref(cfg.c()), batch,
+                                                              max_seq_len, top_k))
+
+
+def decode_step(cfg: LayerConfig, cache: LayerCache, seq_len: torch.Tensor, max_seq_len: int,
+                q: torch.Tensor, kv_new: torch.Tensor, logit_new: torch.Tensor, top_k: int,
+                idx: torch.Tensor | None, cnt: torch.Tensor | None, out: torch.Tensor,
+                workspace: torch.Tensor, status: torch.Tensor, stream=None) -> None:
+    """ckv_decode_step: append the token at seq_len-1, select (top_k > 0) and attend, one call."""
+    batch = int(seq_len.shape[0])
+    _check("ckv_decode_step", load_library().ckv_decode_step(
+        ctypes.byref(cfg.c()), ctypes.byref(cache.c()), batch, _ptr(seq_len), max_seq_len, _ptr(q),
+        _ptr(kv_new), _ptr(logit_new), top_k, _ptr(idx), _ptr(cnt), _ptr(out), _ptr(workspace),
+        workspace.numel(), _ptr(status), _stream(stream)))

@@ -27,6 +27,7 @@ struct AppendArgs {
   const float* kv_new;
   const float* logit_new;
   uint32_t* status;
+  int prev_offset;  // added to prev_len[b]
 };
 
 __device__ float block_max(float v, float* red) {
@@ -254,7 +255,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
   griddep_launch();
   __shared__ float smem[256 + 1024 + 32 + (kAppendThreads / 32) * 1024];
   const int b = blockIdx.y;
-  const int64_t prev = a.prev_len[b];
+  const int64_t prev = static_cast<int64_t>(a.prev_len[b]) + a.prev_offset;
   int64_t row0, n;
   if (a.cu_new) {
     row0 = a.cu_new[b];
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
   const int npairs = p.D / 2;
   const int sp = npairs < kSlicePairs ? npairs : kSlicePairs;
   const int pr_lo = slice * sp;
-  const int64_t prev = a.prev_len[b];
+  const int64_t prev = static_cast<int64_t>(a.prev_len[b]) + a.prev_offset;
   int64_t row0 = b, n = 1;
   if (a.cu_new) {
     row0 = a.cu_new[b];
@@ -469,8 +470,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
 
 cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_len,
                           const int32_t* cu_new, int max_new, int max_seq_len, const float* kv_new,
-                          const float* logit_new, uint32_t* status, cudaStream_t stream) {
-  AppendArgs a{p, prev_len, cu_new, max_seq_len, kv_new, logit_new, status};
+                          const float* logit_new, uint32_t* status, cudaStream_t stream,
+                          int prev_offset) {
+  AppendArgs a{p, prev_len, cu_new, max_seq_len, kv_new, logit_new, status, prev_offset};
   if (max_new == 1) {  // one token per request: the fold split across 64-dim slices
     const int slices = p.D / 2 < kSlicePairs ? 1 : p.D / 2 / kSlicePairs;
     return launch_kernel(append_decode_kernel, dim3(slices, batch), dim3(kAppendThreads), 0, stream, a);

@@ -518,11 +518,14 @@ AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_
 cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq_len,
                              int max_seq_len, const float* q, const int32_t* idx,
                              const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
-                             uint32_t* status, cudaStream_t stream) {
-  const dim3 prep_grid(attention_tc_supported(p) ? 8 : 1, batch);   // 8 heads per CTA on the MMA path
-  cudaError_t e = launch_kernel(attn_prep_kernel, prep_grid, dim3(kPrepThreads), 0, stream, p, seq_len,
-                                max_seq_len, q, ws);
-  if (e != cudaSuccess) return e;
+                             uint32_t* status, cudaStream_t stream, bool prep_done) {
+  cudaError_t e = cudaSuccess;
+  if (!prep_done) {
+    const dim3 prep_grid(attention_tc_supported(p) ? 8 : 1, batch);   // 8 heads per CTA on the MMA path
+    e = launch_kernel(attn_prep_kernel, prep_grid, dim3(kPrepThreads), 0, stream, p, seq_len, max_seq_len,
+                      q, ws);
+    if (e != cudaSuccess) return e;
+  }
   prof_begin(kProfAttention, stream);
   if (attention_tc_supported(p)) {
     e = launch_attention_tc(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);

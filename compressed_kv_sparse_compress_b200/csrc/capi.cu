@@ -293,6 +293,71 @@ int compressed_window_attention(const ckv_layer_cfg* cfg, const ckv_layer_cache*
   return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
 }
 
+// Workspace of a fused step: the indexer's (sparse layers) followed by the attention's, each
+// 256-byte aligned.
+static size_t step_ws_bytes(const LayerParams& p, int batch, int max_seq_len, int top_k, IndexerWs* iw,
+                            AttnWs* aw, void* base) {
+  size_t off = 0;
+  if (top_k > 0) {
+    *iw = indexer_ws_layout(base, p, batch, max_seq_len);
+    off = align_up(iw->bytes, 256);
+  }
+  *aw = attention_ws_layout(base ? static_cast<char*>(base) + off : nullptr, p, batch, max_seq_len,
+                            top_k > 0 ? top_k : 0);
+  return off + aw->bytes;
+}
+
+size_t ckv_decode_step_workspace_bytes(const ckv_layer_cfg* cfg, int32_t batch, int32_t max_seq_len,
+                                       int32_t top_k) {
+  if (check_cfg(cfg) != CKV_OK || batch < 1 || max_seq_len < 1 || top_k < 0) return 0;
+  LayerParams p{};
+  p.H = cfg->num_heads;
+  p.D = cfg->head_dim;
+  p.r = cfg->ratio;
+  p.W = cfg->window;
+  p.comp_dtype = cfg->comp_dtype;
+  p.win_dtype = cfg->win_dtype;
+  p.d_r = cfg->rope_dim;
+  IndexerWs iw{};
+  AttnWs aw{};
+  return step_ws_bytes(p, batch, max_seq_len, top_k, &iw, &aw, nullptr);
+}
+
+int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int32_t batch,
+                    const int32_t* d_seq_len, int32_t max_seq_len, const float* d_q,
+                    const float* d_kv_new, const float* d_logit_new, int32_t top_k, int32_t* d_idx,
+                    int32_t* d_cnt, float* d_out, void* d_ws, size_t ws_bytes, uint32_t* d_status,
+                    void* stream) {
+  LayerParams p{};
+  const int st = make_params(cfg, cache, batch, max_seq_len, true, &p);
+  if (st != CKV_OK) return st;
+  if (batch > 16384) return CKV_ERR_UNSUPPORTED;
+  if (!d_seq_len || !d_q || !d_kv_new || !d_logit_new || !d_out || !d_status || top_k < 0 ||
+      !aligned16(d_q) || !aligned16(d_kv_new) || !aligned16(d_out))
+    return CKV_ERR_INVALID_ARG;
+  if (top_k > 0 && (!d_idx || !d_cnt || !aligned16(d_idx) || !aligned16(d_cnt))) return CKV_ERR_INVALID_ARG;
+  if (!d_ws || !aligned16(d_ws)) return CKV_ERR_WORKSPACE;
+  IndexerWs iw{};
+  AttnWs aw{};
+  if (ws_bytes < step_ws_bytes(p, batch, max_seq_len, top_k, &iw, &aw, d_ws)) return CKV_ERR_WORKSPACE;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the new token of request b is at position seq_len[b] - 1
+  cudaError_t e = launch_append(p, batch, d_seq_len, nullptr, 1, max_seq_len, d_kv_new, d_logit_new, d_status,
+                                s, -1);
+  if (e != cudaSuccess) return CKV_ERR_CUDA;
+  bool prep_done = false;
+  if (top_k > 0) {
+    const QueryPrepOut prep{aw.rope, attention_tc_supported(p) ? aw.qimage : nullptr};
+    e = launch_indexer(p, batch, d_seq_len, max_seq_len, d_q, top_k, d_idx, d_cnt, nullptr, iw, d_status, s,
+                       prep);
+    if (e != cudaSuccess) return CKV_ERR_CUDA;
+    prep_done = true;
+  }
+  e = launch_attention(p, batch, d_seq_len, max_seq_len, d_q, top_k > 0 ? d_idx : nullptr,
+                       top_k > 0 ? d_cnt : nullptr, top_k > 0 ? top_k : 0, d_out, aw, d_status, s, prep_done);
+  return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+}
+
 const char* ckv_status_str(int status) {
   switch (status) {
     case CKV_OK: return "ok";

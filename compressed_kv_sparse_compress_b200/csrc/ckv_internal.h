@@ -43,9 +43,11 @@ void prof_begin(ProfPoint which, cudaStream_t stream);
 void prof_end(ProfPoint which, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------- append
+// prev_offset is added to every prev_len[b] (-1 when prev_len holds the lengths after the append)
 cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_len,
                           const int32_t* cu_new, int max_new, int max_seq_len, const float* kv_new,
-                          const float* logit_new, uint32_t* status, cudaStream_t stream);
+                          const float* logit_new, uint32_t* status, cudaStream_t stream,
+                          int prev_offset = 0);
 
 // ---------------------------------------------------------------------------- indexer
 constexpr int kHistBins = 2048;  // first radix digit: the top 11 bits of the order key
@@ -64,10 +66,16 @@ struct IndexerWs {
 int64_t score_stride(int ratio, int max_seq_len);
 IndexerWs indexer_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len);
 
+// Outputs of the query pass that the attention of the same layer and step can take over (the
+// cos/sin table and, on the tensor-core path, the rotated fp16 query image); null: not written.
+struct QueryPrepOut {
+  double* rope;
+  uint8_t* qimage;
+};
 cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
                            int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
                            float* scores, const IndexerWs& ws, uint32_t* status,
-                           cudaStream_t stream);
+                           cudaStream_t stream, QueryPrepOut prep = {nullptr, nullptr});
 
 // ---------------------------------------------------------------------------- attention
 struct AttnWs {
@@ -85,12 +93,15 @@ struct AttnWs {
   size_t bytes;
 };
 constexpr int kQImageBytes = 64 * 512 * 2;  // H = 64, D = 512 fp16
+bool attention_tc_supported(const LayerParams& p);  // the tensor-core path serves this layer
 AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len,
                            int max_selected);
 
+// prep_done: the cos/sin table and query image are already in ws (written by the indexer's query
+// pass of the same step), so the prep kernel is not launched
 cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq_len,
                              int max_seq_len, const float* q, const int32_t* idx,
                              const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
-                             uint32_t* status, cudaStream_t stream);
+                             uint32_t* status, cudaStream_t stream, bool prep_done = false);
 
 }  // namespace ckv

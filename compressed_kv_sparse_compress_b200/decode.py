@@ -1,7 +1,7 @@
 """One layer of the decode step: append the new token, select, attend.
 
 Owns the per-layer output and workspace buffers so that a decode step is three library calls
-with no allocation. Every step runs in libckv's kernels.
+(or one fused call) with no allocation. Every step runs in libckv's kernels.
 """
 
 from __future__ import annotations
@@ -44,6 +44,7 @@ class DecodeLayer:
             self.idx = self.cnt = self.ws_index = None
         n = B.attention_workspace_bytes(cfg, batch, max_seq_len, top_k or 0)
         self.ws_attn = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+        self.ws_step = None  # fused-step workspace, allocated by the first fused_step
 
     def append(self, prev_len, kv_new, logit_new, cu_new=None, max_new=1, stream=None):
         B.kv_compress_append(self.cfg, self.cache, prev_len, kv_new, logit_new, self.status,
@@ -68,3 +69,13 @@ class DecodeLayer:
         if self.top_k is not None:
             self.select(seq_len, q, stream=stream)
         return self.attend(seq_len, q, stream=stream)
+
+    def fused_step(self, seq_len, q, kv_new, logit_new, stream=None):
+        """The same step as one ckv_decode_step call (its own workspace, allocated once)."""
+        if self.ws_step is None:
+            n = B.decode_step_workspace_bytes(self.cfg, self.batch, self.max_seq_len, self.top_k or 0)
+            self.ws_step = torch.empty(max(n, 16), dtype=torch.uint8, device=self.out.device)
+        B.decode_step(self.cfg, self.cache, seq_len, self.max_seq_len, q, kv_new, logit_new,
+                      self.top_k or 0, self.idx, self.cnt, self.out, self.ws_step, self.status,
+                      stream=stream)
+        return self.out

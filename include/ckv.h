@@ -248,6 +248,34 @@ int sparse_indexer_topk_noalloc(const ckv_layer_cfg* cfg, const ckv_layer_cache*
 /* Diagnostics. */
 
 /* Static text of a ckv_status. */
+/* ---------------------------------------------------------------------------------------- */
+/* Fused decode step of one layer: steps 1-3 in one call (the three descriptions above apply).
+ * [HR] section A lists the path's parts (compression, top-k over compressed tokens, window,
+ * shared K=V attention); [CZ] section C credits the speed-up to fused kernels. One token per
+ * request is appended at position seq_len[b] - 1, the layer's top_k entries are selected
+ * (top_k > 0, CSA) or all entries are attended (top_k == 0, HCA), and the output is written.
+ * Compared with the three calls, the query pass of the indexer also writes the attention's query
+ * preparation (cos/sin table, rotated fp16 query image), so one kernel launch is saved on sparse
+ * layers; every result is bit-identical to the three calls'.
+ *
+ *   d_seq_len    [batch] int32: L_b including the new token (1 .. max_seq_len).
+ *   d_q          [batch][H][D] fp32 raw query; d_kv_new [batch][D] fp32 raw token; d_logit_new
+ *                [batch] fp32 compressor logit.
+ *   top_k        0 for a dense layer; else the selection size, and d_idx [batch][top_k] / d_cnt
+ *                [batch] receive the selection (as sparse_indexer_topk writes it).
+ *   d_out        [batch][H][D] fp32.
+ *   d_ws         workspace of ckv_decode_step_workspace_bytes(cfg, batch, max_seq_len, top_k)
+ *                bytes, 16-byte aligned; its contents need no initialisation.
+ * Errors as for the three calls (host codes before any launch, device status bits after).
+ */
+size_t ckv_decode_step_workspace_bytes(const ckv_layer_cfg* cfg, int32_t batch, int32_t max_seq_len,
+                                       int32_t top_k);
+int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int32_t batch,
+                    const int32_t* d_seq_len, int32_t max_seq_len, const float* d_q,
+                    const float* d_kv_new, const float* d_logit_new, int32_t top_k, int32_t* d_idx,
+                    int32_t* d_cnt, float* d_out, void* d_ws, size_t ws_bytes, uint32_t* d_status,
+                    void* stream);
+
 const char* ckv_status_str(int status);
 /* Number of kernel launches enqueued by this process since load (all entry points). */
 uint64_t ckv_launch_count(void);

@@ -128,3 +128,21 @@ def test_entry_points_reject_null_arguments_before_any_device_work():
     assert st == ckv.CKV_ERR_INVALID_ARG
     assert ckv.status_str(ckv.CKV_ERR_WORKSPACE) == "workspace too small"
     assert ckv.launch_count() == 0
+
+
+def test_fused_step_workspace_and_argument_checks():
+    cfg = ckv.LayerConfig(64, 512, 64, 4, 128, "bf16", "fp8")
+    sparse = ckv.decode_step_workspace_bytes(cfg, 8, 32768, 512)
+    dense = ckv.decode_step_workspace_bytes(cfg, 8, 32768, 0)
+    # the fused step's workspace holds the indexer's and the attention's, each 256-byte aligned
+    assert sparse >= ckv.indexer_workspace_bytes(cfg, 8, 32768, 512) + ckv.attention_workspace_bytes(cfg, 8, 32768, 512)
+    assert dense == ckv.attention_workspace_bytes(cfg, 8, 32768, 0)
+    assert ckv.decode_step_workspace_bytes(cfg, 8, 32768, -1) == 0
+    bad = ckv.LayerConfig(8, 100, 32, 4, 128, "bf16", "fp8")
+    assert ckv.decode_step_workspace_bytes(bad, 1, 1024, 16) == 0
+    lib = ckv.load_library()
+    cache = ckv.LayerCacheC()  # all NULL
+    st = lib.ckv_decode_step(ctypes.byref(cfg.c()), ctypes.byref(cache), 1, None, 1024, None, None, None, 4,
+                             None, None, None, None, 0, None, None)
+    assert st == ckv.CKV_ERR_INVALID_ARG
+    assert ckv.launch_count() == 0

@@ -1,0 +1,72 @@
+"""ckv_decode_step: append, select and attend of one layer in one call.
+
+The fused call runs the same kernels as the three calls except that the indexer's query pass also
+writes the attention's query preparation (cos/sin table and, for H = 64 and D = 512, the rotated
+fp16 query image) with the prep kernel's arithmetic, so every result must be bit-identical to the
+three calls': the output, the selection and every byte the append writes. Each side works on its
+own copy of the same generated pools.
+"""
+
+import pytest
+import torch
+
+from synth import workloads as S
+from tests import ckv_testlib as T
+
+pytestmark = pytest.mark.gpu
+
+CACHE_PLANES = ("comp_codes", "comp_scales", "win_codes", "win_scales", "residue_kv", "residue_logit")
+
+SMALL = [
+    S.scaled(S.csa_b8_ctx32k(), (32768, 20001, 4099, 9, 700, 131), "fused", seed=6000),
+    S.scaled(S.hca_b32_ctx128k(), (131072, 60000, 129, 1000), "fused", seed=6001),
+    S.scaled(S.mixed_64req(), (16385, 5000, 1025, 70000), "fused", seed=6002),
+    S.csa_b1_ctx4k_fp32(),
+]
+
+
+def _bytes(t):
+    return t.contiguous().view(torch.uint8)
+
+
+def _check_fused_equals_three_calls(cuda_lib, w):
+    gen = S.generate(w, "cuda")
+    seq = gen["seq_len"]
+    for li, (lay, ls) in enumerate(zip(gen["layers"], w.layers)):
+        three = T.gpu_layer(cuda_lib, w, lay, ls)
+        fused = T.gpu_layer(cuda_lib, w, lay, ls)
+        T.gpu_setup(three, lay)
+        T.gpu_setup(fused, lay)
+        out3 = three.step(seq, (seq - 1).to(torch.int32), lay["q"], lay["kv_new"], lay["logit_new"]).clone()
+        out1 = fused.fused_step(seq, lay["q"], lay["kv_new"], lay["logit_new"]).clone()
+        assert T.status_word(three) == 0 and T.status_word(fused) == 0
+        assert torch.equal(_bytes(out1), _bytes(out3)), f"{w.name} layer {li}: outputs differ"
+        if ls.top_k is not None:
+            assert torch.equal(fused.cnt, three.cnt)
+            assert torch.equal(fused.idx, three.idx)
+        for name in CACHE_PLANES:
+            a, b = getattr(three.cache, name), getattr(fused.cache, name)
+            if a is not None:
+                assert torch.equal(_bytes(a), _bytes(b)), f"{w.name} layer {li}: {name} differs"
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_fused_step_is_bit_identical_to_the_three_calls(cuda_lib, w):
+    _check_fused_equals_three_calls(cuda_lib, w)
+
+
+def test_fused_step_at_full_size(cuda_lib):
+    _check_fused_equals_three_calls(cuda_lib, S.csa_b8_ctx32k())
+    torch.cuda.empty_cache()
+
+
+def test_fused_step_sets_the_status_of_a_bad_length(cuda_lib):
+    w = SMALL[0]
+    gen = S.generate(w, "cuda")
+    lay, ls = gen["layers"][0], w.layers[0]
+    dl = T.gpu_layer(cuda_lib, w, lay, ls)
+    seq = gen["seq_len"].clone()
+    seq[2] = max(w.seq_lens) + 5  # above max_seq_len: flagged, that request skipped
+    out = dl.fused_step(seq, lay["q"], lay["kv_new"], lay["logit_new"])
+    assert T.status_word(dl) & cuda_lib.CKV_DEV_BAD_LENGTH
+    assert torch.count_nonzero(out[2]) == 0
