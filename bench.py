@@ -329,8 +329,8 @@ def run_cuda(args, w: S.Workload):
         seq_d.copy_(seq_h, non_blocking=True)
         for a, b in zip(q_d + kv_d + lg_d, q_h + kv_h + lg_h):
             a.copy_(b, non_blocking=True)
-        prev_d = seq_d - 1
-        outs = step.run(q_d, kv_d, lg_d, seq_d, prev_d.to(torch.int32))
+        prev_d = (seq_d - 1).to(torch.int32) if step.api == "calls" else None
+        outs = step.run(q_d, kv_d, lg_d, seq_d, prev_d)
         for o, oh in zip(outs, out_h):
             oh.copy_(o, non_blocking=True)
 
@@ -338,12 +338,26 @@ def run_cuda(args, w: S.Workload):
         flush_l2()
         e2e_step()
     barrier()
+    # the whole end-to-end step (copies in, every layer's call, copy out) as one CUDA graph
+    run_e2e, graph_note = e2e_step, "eager"
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                e2e_step()
+            graph.replay()
+            torch.cuda.synchronize()
+            run_e2e, graph_note = graph.replay, "one CUDA graph per step (copies and kernels)"
+        except RuntimeError as exc:   # capture refused: stay eager and say so
+            graph_note = "eager (graph capture failed: %s)" % str(exc).splitlines()[0][:120]
+            torch.cuda.synchronize()
     eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    barrier()
     for i in range(args.steps):
         flush_l2()
         eev[i][0].record(stream)
-        e2e_step()
+        run_e2e()
         eev[i][1].record(stream)
     barrier()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev), dev)
@@ -388,7 +402,7 @@ def run_cuda(args, w: S.Workload):
                                  "of the kernel (that pass: %.1f us per step)" % (kstep_ms / args.steps * 1e3),
                      "traffic": traffic_record(dominant, w.name)},
         "e2e": {"value": job_throughput(w.batch * len(w.layers), ws, args.steps, e2e_ms), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "launch": graph_note,
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": launches,
         "clocks": clk,
@@ -513,6 +527,7 @@ def main():
                     help="fused: one ckv_decode_step per layer; calls: append, select, attend")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="end-to-end steps launched eagerly")
     ap.add_argument("--reference-requests", type=int, default=0,
                     help="requests of the batch the reference arm runs per step (0: all)")
     args = ap.parse_args()

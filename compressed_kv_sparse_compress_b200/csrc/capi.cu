@@ -37,9 +37,25 @@ int sm_count() {
   return cache[dev];
 }
 
+// Raises a kernel's dynamic shared-memory limit once per (device, kernel, larger size); later calls
+// with the same or a smaller size make no CUDA call (so they are free inside graph capture too).
 cudaError_t allow_smem(const void* kernel, int bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  struct Entry {
+    int dev;
+    const void* kernel;
+    int bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  for (Entry& e : done)
+    if (e.dev == dev && e.kernel == kernel && e.bytes >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back({dev, kernel, bytes});
+  return e;
 }
 
 namespace {
