@@ -711,15 +711,22 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
     const uint2 r2 = small_boundary<4>(c2, need2, wsum[1], &bnd);
     const uint32_t need3 = need2 - r2.y;
     const uint32_t p2 = (r1.x << 11) | r2.x;
+    if (h2[r2.x] == need3 && p2 > 0) {
+      // every key of the boundary bin is taken: the threshold is the bin's lower edge (the same
+      // in every thread; the last digit is not needed)
+      T = (p2 << 10) - 1;
+      quota = 0;
+    } else {
 #pragma unroll
-    for (int u = 0; u < kSmallPerThread; ++u)
-      if (((valid >> u) & 1u) && (key[u] >> 10) == p2) atomicAdd(h3 + (key[u] & 1023u), 1u);
-    __syncthreads();
-    const uint2 c3v = reinterpret_cast<const uint2*>(h3)[tid];
-    const uint32_t c3[2] = {c3v.x, c3v.y};
-    const uint2 r3 = small_boundary<2>(c3, need3, wsum[0], &bnd);
-    T = (p2 << 10) | r3.x;
-    quota = need3 - r3.y;
+      for (int u = 0; u < kSmallPerThread; ++u)
+        if (((valid >> u) & 1u) && (key[u] >> 10) == p2) atomicAdd(h3 + (key[u] & 1023u), 1u);
+      __syncthreads();
+      const uint2 c3v = reinterpret_cast<const uint2*>(h3)[tid];
+      const uint32_t c3[2] = {c3v.x, c3v.y};
+      const uint2 r3 = small_boundary<2>(c3, need3, wsum[0], &bnd);
+      T = (p2 << 10) | r3.x;
+      quota = need3 - r3.y;
+    }
   }
 
   // one exclusive block scan of (count above T) << 16 | (count equal to T), both <= kSmallMax
