@@ -12,6 +12,7 @@
 // group of the call is made of new tokens only and is handled by any block, grid-strided.
 
 #include "ckv_internal.h"
+#include "query_prep.cuh"
 
 namespace ckv {
 namespace {
@@ -296,16 +297,38 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
 constexpr int kSlicePairs = 32;
 constexpr int kRingPreload = 16;  // ring tokens per warp whose loads are issued at the start
 
-__global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArgs a) {
-  griddep_wait();
-  griddep_launch();
-  __shared__ float w[256];
-  __shared__ float2 part[kAppendThreads / 32][kSlicePairs];
-  __shared__ float2 xs[kSlicePairs];
-  __shared__ float c[2 * kSlicePairs];
-  __shared__ float red[32];
+// Shared memory of one append_decode_slice group.
+struct AppendDecodeSmem {
+  float w[256];
+  float2 part[kAppendThreads / 32][kSlicePairs];
+  float2 xs[kSlicePairs];
+  float c[2 * kSlicePairs];
+  float red[32];
+};
+
+// max over a group of 256 threads (ids tid) synchronising through barrier bar_id
+__device__ float group_max(float v, float* red, int tid, int bar_id) {
+  v = warp_max(v);
+  const int w = tid >> 5, l = tid & 31;
+  group_sync(bar_id);
+  if (l == 0) red[w] = v;
+  group_sync(bar_id);
+  float m = (tid < kAppendThreads / 32) ? red[tid] : 0.f;
+  if (w == 0) m = warp_max(m);
+  if (tid == 0) red[0] = m;
+  group_sync(bar_id);
+  return red[0];
+}
+
+// Slice `slice` of request b, on a group of 256 threads (ids tid, barrier bar_id).
+__device__ void append_decode_slice(const AppendArgs& a, int slice, int b, int tid, int bar_id,
+                                    AppendDecodeSmem& sm) {
+  float* w = sm.w;
+  float2 (*part)[kSlicePairs] = sm.part;
+  float2* xs = sm.xs;
+  float* c = sm.c;
+  float* red = sm.red;
   const LayerParams& p = a.p;
-  const int b = blockIdx.y, slice = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, nw = kAppendThreads / 32;
   const int npairs = p.D / 2;
   const int sp = npairs < kSlicePairs ? npairs : kSlicePairs;
@@ -376,7 +399,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
 #pragma unroll
       for (int k = 0; k < kMaxPairsPerThread; ++k)
         amax = fmaxf(amax, fmaxf(fabsf(x[k].x), fabsf(x[k].y)));  // zero beyond npairs
-      amax = block_max(amax, red);
+      amax = group_max(amax, red, tid, bar_id);
       if (wrow >= 0) {
         const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
         uint16_t* dst = reinterpret_cast<uint16_t*>(p.win_codes + wrow * p.win_row_bytes);
@@ -395,7 +418,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
   if (!complete) return;
 
   // softmax weights of the group
-  __syncthreads();
+  group_sync(bar_id);
   if (warp == 0) {
     float m = -INFINITY;
     for (int t = lane; t < r; t += 32) m = fmaxf(m, w[t]);
@@ -409,7 +432,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
     sum = warp_sum(sum);
     for (int t = lane; t < r; t += 32) w[t] = w[t] / sum;
   }
-  __syncthreads();
+  group_sync(bar_id);
   // ring tokens: warp partial sums over its run of tokens, lane = pair of the slice
   float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
@@ -425,7 +448,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
     acc.y = fmaf(w[t], v.y, acc.y);
   }
   if (lane < sp) part[warp][lane] = acc;
-  __syncthreads();
+  group_sync(bar_id);
   if (tid < sp) {
     float2 e = make_float2(0.f, 0.f);
     for (int ww = 0; ww < nw; ++ww) {
@@ -437,7 +460,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
     c[2 * tid] = e.x;
     c[2 * tid + 1] = e.y;
   }
-  __syncthreads();
+  group_sync(bar_id);
   if (crow < 0) return;
   // this slice's dims of the entry
   const int d_lo = 2 * pr_lo, nd = 2 * sp;
@@ -466,7 +489,57 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
   }
 }
 
+__global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArgs a) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ AppendDecodeSmem sm;
+  append_decode_slice(a, blockIdx.x, blockIdx.y, threadIdx.x, 0, sm);
+}
+
+// ---------------------------------------------------------------------------- fused step front
+
+// First kernel of a fused decode step: the append of one slice (threads 0..255) and, on the other
+// 256 threads, the query pass of the same step (q_bar plus the attention's query preparation on
+// sparse layers, the query preparation alone on dense ones), which reads only the query. The two
+// halves synchronise on barriers 1 and 2 and never wait for each other.
+template <bool kSparse>
+__global__ void __launch_bounds__(2 * kAppendThreads, 1) step_front_kernel(
+    AppendArgs a, int app_slices, const float* q, IndexerWs iws, QueryPrepOut prep, AttnWs aws,
+    int prep_parts) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ AppendDecodeSmem sm;
+  __shared__ double qsm[1024];  // q_bar partial sums [256][2] or the cos/sin table [512][2]
+  const int x = blockIdx.x, b = blockIdx.y;
+  if (threadIdx.x < kAppendThreads) {
+    if (x < app_slices) append_decode_slice(a, x, b, threadIdx.x, 1, sm);
+  } else if (kSparse) {
+    if (x < kQbarSlices)
+      qbar_slice(a.p, a.prev_len, a.max_seq_len, q, iws, a.status, prep, x, b, threadIdx.x - kAppendThreads,
+                 reinterpret_cast<double(*)[2]>(qsm), 2);
+  } else if (x < prep_parts) {
+    prep_part(a.p, a.prev_len, a.max_seq_len, q, aws, x, b, threadIdx.x - kAppendThreads, qsm, 2);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_step_front(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
+                              const float* kv_new, const float* logit_new, const float* q, bool sparse,
+                              const IndexerWs& iws, QueryPrepOut prep, const AttnWs& aws,
+                              uint32_t* status, cudaStream_t stream) {
+  // the new token of request b is at position seq_len[b] - 1
+  const AppendArgs a{p, seq_len, nullptr, max_seq_len, kv_new, logit_new, status, -1};
+  const int app_slices = p.D / 2 < kSlicePairs ? 1 : p.D / 2 / kSlicePairs;
+  const int prep_parts = attention_tc_supported(p) ? 8 : 1;
+  const int other = sparse ? kQbarSlices : prep_parts;
+  const dim3 grid(app_slices > other ? app_slices : other, batch);
+  if (sparse)
+    return launch_kernel(step_front_kernel<true>, grid, dim3(2 * kAppendThreads), 0, stream, a, app_slices, q,
+                         iws, prep, aws, prep_parts);
+  return launch_kernel(step_front_kernel<false>, grid, dim3(2 * kAppendThreads), 0, stream, a, app_slices, q,
+                       iws, prep, aws, prep_parts);
+}
 
 cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_len,
                           const int32_t* cu_new, int max_new, int max_seq_len, const float* kv_new,

@@ -15,6 +15,7 @@
 // combine. The tensor-core path for H=64 lives in attention_tc.cu and writes the same partials.
 
 #include "ckv_internal.h"
+#include "query_prep.cuh"
 #include "ckv_ptx.cuh"
 
 namespace ckv {
@@ -159,76 +160,14 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   }
 }
 
-// Per request: cos/sin of every rotary pair at the query position L-1 (fp64 angles), for the
-// inverse rotation in the combine; on the tensor-core path also the rotated query rounded to
-// fp16, written as the 128-byte-swizzled image of the MMA operand so that each attention CTA
-// fetches it with one bulk copy.
-constexpr int kPrepThreads = 256;
-
+// Query preparation of one part of one request: prep_part (query_prep.cuh).
 __global__ void __launch_bounds__(kPrepThreads) attn_prep_kernel(LayerParams p, const int32_t* seq_len,
                                                                  int max_seq_len, const float* q,
                                                                  AttnWs ws) {
   griddep_wait();
   griddep_launch();
   __shared__ double rope_s[2 * 512];
-  const int b = blockIdx.y;
-  const int L = seq_len[b];
-  if (L < 1 || L > max_seq_len) return;
-  const int n_pairs = p.d_r / 2;
-  double* rope_g = ws.rope + static_cast<int64_t>(b) * (n_pairs + 1) * 2;
-  for (int i = threadIdx.x; i < n_pairs; i += blockDim.x) {
-    double sn, cs;
-    sincos(static_cast<double>(L - 1) * rope_inv_freq(p, i), &sn, &cs);
-    rope_s[2 * i] = cs;
-    rope_s[2 * i + 1] = sn;
-    if (blockIdx.x == 0) {
-      rope_g[2 * i] = cs;
-      rope_g[2 * i + 1] = sn;
-    }
-  }
-  if (!ws.qimage) return;
-  __syncthreads();
-  // tensor-core path (H = 64, D = 512): granule g (8 dims) of head h lands at chunk g/8, row h,
-  // 16-byte slot (g % 8) ^ (h % 8) of the operand image; CTA x builds heads 8x .. 8x+7
-  constexpr int kD = 512, kGr = kD / 8, kChunk = 64 * 128;
-  const float* qb = q + static_cast<int64_t>(b) * 64 * kD;
-  uint8_t* img = ws.qimage + static_cast<int64_t>(b) * kQImageBytes;
-  const int first_rope = (kD - p.d_r) / 2;
-  for (int it0 = blockIdx.x * 8 * kGr; it0 < (blockIdx.x + 1) * 8 * kGr; it0 += 2 * kPrepThreads) {
-    float4 raw[2][2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int it = it0 + u * kPrepThreads + threadIdx.x;
-      const float4* src = reinterpret_cast<const float4*>(qb + (it >> 6) * kD + 8 * (it & 63));
-      raw[u][0] = __ldg(src);
-      raw[u][1] = __ldg(src + 1);
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int it = it0 + u * kPrepThreads + threadIdx.x;
-      const int h = it >> 6, g = it & 63;
-      float v[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
-                    raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int pr = 4 * g + k;
-        if (pr >= first_rope) {
-          const double cs = rope_s[2 * (pr - first_rope)], sn = rope_s[2 * (pr - first_rope) + 1];
-          const double x0 = v[2 * k], x1 = v[2 * k + 1];
-          v[2 * k] = static_cast<float>(x0 * cs - x1 * sn);
-          v[2 * k + 1] = static_cast<float>(x0 * sn + x1 * cs);
-        }
-      }
-      uint32_t w[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        __half2 hh = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
-        w[k] = *reinterpret_cast<uint32_t*>(&hh);
-      }
-      const uint32_t off = static_cast<uint32_t>(g >> 3) * kChunk + h * 128 + (((g & 7) ^ (h & 7)) << 4);
-      *reinterpret_cast<uint4*>(img + off) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  }
+  prep_part(p, seq_len, max_seq_len, q, ws, blockIdx.x, blockIdx.y, threadIdx.x, rope_s, 0);
 }
 
 // Merge of the splits of one (request, head) and inverse rotation for the CUDA-core path (fp32

@@ -357,20 +357,19 @@ int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int3
   AttnWs aw{};
   if (ws_bytes < step_ws_bytes(p, batch, max_seq_len, top_k, &iw, &aw, d_ws)) return CKV_ERR_WORKSPACE;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the new token of request b is at position seq_len[b] - 1
-  cudaError_t e = launch_append(p, batch, d_seq_len, nullptr, 1, max_seq_len, d_kv_new, d_logit_new, d_status,
-                                s, -1);
+  // append of the token at seq_len[b] - 1 side by side with the query pass (q_bar and the
+  // attention's query preparation), then selection (sparse layers) and attention
+  const QueryPrepOut prep{aw.rope, attention_tc_supported(p) ? aw.qimage : nullptr};
+  cudaError_t e = launch_step_front(p, batch, d_seq_len, max_seq_len, d_kv_new, d_logit_new, d_q, top_k > 0,
+                                    iw, prep, aw, d_status, s);
   if (e != cudaSuccess) return CKV_ERR_CUDA;
-  bool prep_done = false;
   if (top_k > 0) {
-    const QueryPrepOut prep{aw.rope, attention_tc_supported(p) ? aw.qimage : nullptr};
     e = launch_indexer(p, batch, d_seq_len, max_seq_len, d_q, top_k, d_idx, d_cnt, nullptr, iw, d_status, s,
-                       prep);
+                       prep, true);
     if (e != cudaSuccess) return CKV_ERR_CUDA;
-    prep_done = true;
   }
   e = launch_attention(p, batch, d_seq_len, max_seq_len, d_q, top_k > 0 ? d_idx : nullptr,
-                       top_k > 0 ? d_cnt : nullptr, top_k > 0 ? top_k : 0, d_out, aw, d_status, s, prep_done);
+                       top_k > 0 ? d_cnt : nullptr, top_k > 0 ? top_k : 0, d_out, aw, d_status, s, true);
   return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
 }
 

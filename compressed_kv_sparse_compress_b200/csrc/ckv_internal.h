@@ -72,10 +72,13 @@ struct QueryPrepOut {
   double* rope;
   uint8_t* qimage;
 };
+// skip_qbar: q_bar, the counts and the reset of the selection state are already done (by the
+// fused step's front kernel)
 cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
                            int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
                            float* scores, const IndexerWs& ws, uint32_t* status,
-                           cudaStream_t stream, QueryPrepOut prep = {nullptr, nullptr});
+                           cudaStream_t stream, QueryPrepOut prep = {nullptr, nullptr},
+                           bool skip_qbar = false);
 
 // ---------------------------------------------------------------------------- attention
 struct AttnWs {
@@ -103,5 +106,14 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
                              int max_seq_len, const float* q, const int32_t* idx,
                              const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
                              uint32_t* status, cudaStream_t stream, bool prep_done = false);
+
+// ---------------------------------------------------------------------------- fused step
+// First kernel of ckv_decode_step: the append of the new token (at seq_len[b] - 1) side by side
+// with the query pass (q_bar and the query preparation on sparse layers, the preparation alone on
+// dense ones).
+cudaError_t launch_step_front(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
+                              const float* kv_new, const float* logit_new, const float* q, bool sparse,
+                              const IndexerWs& iws, QueryPrepOut prep, const AttnWs& aws,
+                              uint32_t* status, cudaStream_t stream);
 
 }  // namespace ckv

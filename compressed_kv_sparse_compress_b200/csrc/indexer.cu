@@ -22,6 +22,7 @@
 //                   lower-index tie rule), then compacts the bitmap into ascending indices.
 
 #include "ckv_internal.h"
+#include "query_prep.cuh"
 
 namespace ckv {
 
@@ -130,17 +131,7 @@ __device__ void find_boundary(const uint32_t* h, int nbins, uint32_t need, bool 
 
 // ---------------------------------------------------------------------------- q_bar
 
-// kQbarSlices CTAs of 256 threads per request, CTA s owning the rotary-aligned dim pairs
-// [s * P, (s + 1) * P) with P = D / 2 / kQbarSlices: thread (pair k, head group g) sums its heads of
-// one pair in fp64 with all its loads in flight at once; the head groups are added in shared
-// memory, the sum rotated and scaled. The slices also reset the request's selection state.
-// With `prep` set (a fused decode step), the same pass writes what the attention's query
-// preparation would: the cos/sin table of the rotary pairs and, for H = 64 and D = 512, every
-// head's rotated query rounded to fp16 in the swizzled operand layout (chunk of 64 dims = slice,
-// row = head), with the prep kernel's arithmetic.
-constexpr int kQbarThreads = 256;
-constexpr int kQbarSlices = 8;
-
+// q_bar of one slice of one request: qbar_slice (query_prep.cuh).
 __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const int32_t* seq_len,
                                                             int max_seq_len, const float* q,
                                                             IndexerWs ws, uint32_t* status,
@@ -148,85 +139,7 @@ __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const
   griddep_wait();
   griddep_launch();
   __shared__ double part[kQbarThreads][2];
-  const int b = blockIdx.y, slice = blockIdx.x, tid = threadIdx.x;
-  const int L = seq_len[b];
-  const bool ok = L >= 1 && L <= max_seq_len;
-  if (slice == 0 && tid == 0) {
-    if (!ok) atomicOr(status, CKV_DEV_BAD_LENGTH);
-    ws.n_c[b] = ok ? L / p.r : 0;
-    ws.cand_cnt[b] = 0;
-  }
-  constexpr int kBinsPerSlice = kHistBins / kQbarSlices;
-  for (int i = tid; i < kBinsPerSlice; i += kQbarThreads)
-    ws.hist[static_cast<int64_t>(b) * kHistBins + slice * kBinsPerSlice + i] = 0;
-  const int P = p.D / 2 / kQbarSlices;  // 4 .. 64 pairs (D = 64 .. 1024)
-  const int G = kQbarThreads / P;       // head groups
-  const int k = tid % P, g = tid / P;
-  const int pr = slice * P + k, first_rope = (p.D - p.d_r) / 2;
-  const float* qb = q + static_cast<int64_t>(b) * p.H * p.D;
-  const int h_lo = (p.H * g) / G, h_hi = (p.H * (g + 1)) / G;
-  const bool rope_pair = pr >= first_rope && ok;
-  const bool image = prep.qimage != nullptr && ok;  // H = 64, D = 512 (checked by the caller)
-  const bool rotate = rope_pair && (g == 0 || image);
-  double s0 = 0.0, s1 = 0.0, rsn = 0.0, rcs = 1.0;
-  bool have_angle = false;
-  for (int h0 = h_lo; h0 < h_hi; h0 += 16) {
-    float2 v[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u)
-      v[u] = h0 + u < h_hi ? __ldg(reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h0 + u) * p.D) + pr)
-                           : make_float2(0.f, 0.f);
-    if (rotate && !have_angle) {  // rotation angle while the loads fly
-      sincos(static_cast<double>(L - 1) * rope_inv_freq(p, pr - first_rope), &rsn, &rcs);
-      have_angle = true;
-    }
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      s0 += v[u].x;
-      s1 += v[u].y;
-    }
-    if (image) {  // head h0 + u, dims 2pr, 2pr + 1 -> chunk pr/32, row h, slot ((pr%32)/4)^(h%8), word pr%4
-      uint8_t* img = prep.qimage + static_cast<int64_t>(b) * kQImageBytes + (pr >> 5) * (64 * 128) + (pr & 3) * 4;
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int h = h0 + u;
-        if (h >= h_hi) break;
-        float x0 = v[u].x, x1 = v[u].y;
-        if (rope_pair) {
-          const double a0 = x0, a1 = x1;
-          x0 = static_cast<float>(a0 * rcs - a1 * rsn);
-          x1 = static_cast<float>(a0 * rsn + a1 * rcs);
-        }
-        const __half2 hh = __floats2half2_rn(x0, x1);
-        *reinterpret_cast<__half2*>(img + h * 128 + ((((pr & 31) >> 2) ^ (h & 7)) << 4)) = hh;
-      }
-    }
-  }
-  if (rotate && !have_angle)  // head group 0 holds no heads when H < G
-    sincos(static_cast<double>(L - 1) * rope_inv_freq(p, pr - first_rope), &rsn, &rcs);
-  if (prep.rope && rope_pair && g == 0) {
-    double* rope_g = prep.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
-    rope_g[2 * (pr - first_rope)] = rcs;
-    rope_g[2 * (pr - first_rope) + 1] = rsn;
-  }
-  part[tid][0] = s0;
-  part[tid][1] = s1;
-  __syncthreads();
-  if (g == 0) {
-    double a = 0.0, c = 0.0;
-    for (int gg = 0; gg < G; ++gg) {
-      a += part[gg * P + k][0];
-      c += part[gg * P + k][1];
-    }
-    if (rope_pair) {
-      const double x = a;
-      a = x * rcs - c * rsn;
-      c = x * rsn + c * rcs;
-    }
-    const double scale = static_cast<double>(p.sm_scale) / p.H;
-    reinterpret_cast<float2*>(ws.qbar + static_cast<int64_t>(b) * p.D)[pr] =
-        make_float2(static_cast<float>(a * scale), static_cast<float>(c * scale));
-  }
+  qbar_slice(p, seq_len, max_seq_len, q, ws, status, prep, blockIdx.x, blockIdx.y, threadIdx.x, part, 0);
 }
 
 // ---------------------------------------------------------------------------- scoring
@@ -826,12 +739,15 @@ cudaError_t dispatch_score(const LayerParams& p, int batch, int max_seq_len, con
 cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
                            int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
                            float* scores, const IndexerWs& ws, uint32_t* status,
-                           cudaStream_t stream, QueryPrepOut prep) {
+                           cudaStream_t stream, QueryPrepOut prep, bool skip_qbar) {
   const int64_t stride = score_stride(p.r, max_seq_len);
   float* sc = scores ? scores : ws.scores;
-  cudaError_t e = launch_kernel(qbar_kernel, dim3(kQbarSlices, batch), dim3(kQbarThreads), 0, stream, p, seq_len,
-                                max_seq_len, q, ws, status, prep);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!skip_qbar) {
+    e = launch_kernel(qbar_kernel, dim3(kQbarSlices, batch), dim3(kQbarThreads), 0, stream, p, seq_len,
+                      max_seq_len, q, ws, status, prep);
+    if (e != cudaSuccess) return e;
+  }
   switch (p.comp_dtype) {
     case CKV_F32: e = dispatch_score<CKV_F32>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
     case CKV_BF16: e = dispatch_score<CKV_BF16>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;

@@ -1,0 +1,182 @@
+// Query passes shared by the kernels of the indexer, the attention and the fused decode step's
+// front kernel: the head-averaged query q_bar of the indexer (one slice of dim pairs per call)
+// and the attention's query preparation (cos/sin table, rotated fp16 operand image). Each runs on
+// a group of 256 threads (ids tid) that synchronise through barrier bar_id (0 when the group is
+// the whole CTA).
+#pragma once
+
+#include "ckv_internal.h"
+
+namespace ckv {
+
+constexpr int kQbarThreads = 256;
+constexpr int kQbarSlices = 8;
+constexpr int kPrepThreads = 256;
+
+__device__ __forceinline__ void group_sync(int bar_id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(256) : "memory");
+}
+
+// kQbarSlices CTAs of 256 threads per request, CTA s owning the rotary-aligned dim pairs
+// [s * P, (s + 1) * P) with P = D / 2 / kQbarSlices: thread (pair k, head group g) sums its heads of
+// one pair in fp64 with all its loads in flight at once; the head groups are added in shared
+// memory, the sum rotated and scaled. The slices also reset the request's selection state.
+// With `prep` set (a fused decode step), the same pass writes what the attention's query
+// preparation would: the cos/sin table of the rotary pairs and, for H = 64 and D = 512, every
+// head's rotated query rounded to fp16 in the swizzled operand layout (chunk of 64 dims = slice,
+// row = head), with the prep kernel's arithmetic.
+
+__device__ __forceinline__ void qbar_slice(const LayerParams& p, const int32_t* seq_len, int max_seq_len,
+                                           const float* q, const IndexerWs& ws, uint32_t* status,
+                                           const QueryPrepOut& prep, int slice, int b, int tid,
+                                           double (*part)[2], int bar_id) {
+  const int L = seq_len[b];
+  const bool ok = L >= 1 && L <= max_seq_len;
+  if (slice == 0 && tid == 0) {
+    if (!ok) atomicOr(status, CKV_DEV_BAD_LENGTH);
+    ws.n_c[b] = ok ? L / p.r : 0;
+    ws.cand_cnt[b] = 0;
+  }
+  constexpr int kBinsPerSlice = kHistBins / kQbarSlices;
+  for (int i = tid; i < kBinsPerSlice; i += kQbarThreads)
+    ws.hist[static_cast<int64_t>(b) * kHistBins + slice * kBinsPerSlice + i] = 0;
+  const int P = p.D / 2 / kQbarSlices;  // 4 .. 64 pairs (D = 64 .. 1024)
+  const int G = kQbarThreads / P;       // head groups
+  const int k = tid % P, g = tid / P;
+  const int pr = slice * P + k, first_rope = (p.D - p.d_r) / 2;
+  const float* qb = q + static_cast<int64_t>(b) * p.H * p.D;
+  const int h_lo = (p.H * g) / G, h_hi = (p.H * (g + 1)) / G;
+  const bool rope_pair = pr >= first_rope && ok;
+  const bool image = prep.qimage != nullptr && ok;  // H = 64, D = 512 (checked by the caller)
+  const bool rotate = rope_pair && (g == 0 || image);
+  double s0 = 0.0, s1 = 0.0, rsn = 0.0, rcs = 1.0;
+  bool have_angle = false;
+  for (int h0 = h_lo; h0 < h_hi; h0 += 16) {
+    float2 v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      v[u] = h0 + u < h_hi ? __ldg(reinterpret_cast<const float2*>(qb + static_cast<int64_t>(h0 + u) * p.D) + pr)
+                           : make_float2(0.f, 0.f);
+    if (rotate && !have_angle) {  // rotation angle while the loads fly
+      sincos(static_cast<double>(L - 1) * rope_inv_freq(p, pr - first_rope), &rsn, &rcs);
+      have_angle = true;
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      s0 += v[u].x;
+      s1 += v[u].y;
+    }
+    if (image) {  // head h0 + u, dims 2pr, 2pr + 1 -> chunk pr/32, row h, slot ((pr%32)/4)^(h%8), word pr%4
+      uint8_t* img = prep.qimage + static_cast<int64_t>(b) * kQImageBytes + (pr >> 5) * (64 * 128) + (pr & 3) * 4;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int h = h0 + u;
+        if (h >= h_hi) break;
+        float x0 = v[u].x, x1 = v[u].y;
+        if (rope_pair) {
+          const double a0 = x0, a1 = x1;
+          x0 = static_cast<float>(a0 * rcs - a1 * rsn);
+          x1 = static_cast<float>(a0 * rsn + a1 * rcs);
+        }
+        const __half2 hh = __floats2half2_rn(x0, x1);
+        *reinterpret_cast<__half2*>(img + h * 128 + ((((pr & 31) >> 2) ^ (h & 7)) << 4)) = hh;
+      }
+    }
+  }
+  if (rotate && !have_angle)  // head group 0 holds no heads when H < G
+    sincos(static_cast<double>(L - 1) * rope_inv_freq(p, pr - first_rope), &rsn, &rcs);
+  if (prep.rope && rope_pair && g == 0) {
+    double* rope_g = prep.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
+    rope_g[2 * (pr - first_rope)] = rcs;
+    rope_g[2 * (pr - first_rope) + 1] = rsn;
+  }
+  part[tid][0] = s0;
+  part[tid][1] = s1;
+  group_sync(bar_id);
+  if (g == 0) {
+    double a = 0.0, c = 0.0;
+    for (int gg = 0; gg < G; ++gg) {
+      a += part[gg * P + k][0];
+      c += part[gg * P + k][1];
+    }
+    if (rope_pair) {
+      const double x = a;
+      a = x * rcs - c * rsn;
+      c = x * rsn + c * rcs;
+    }
+    const double scale = static_cast<double>(p.sm_scale) / p.H;
+    reinterpret_cast<float2*>(ws.qbar + static_cast<int64_t>(b) * p.D)[pr] =
+        make_float2(static_cast<float>(a * scale), static_cast<float>(c * scale));
+  }
+}
+
+// Per request: cos/sin of every rotary pair at the query position L-1 (fp64 angles), for the
+// inverse rotation in the combine; on the tensor-core path also the rotated query rounded to
+// fp16, written as the 128-byte-swizzled image of the MMA operand so that each attention CTA
+// fetches it with one bulk copy.
+
+// Part `part` of request b (part 0 alone on the CUDA-core path; parts 0..7 build heads 8x .. 8x+7
+// of the tensor-core image), kPrepThreads threads with ids tid.
+__device__ __forceinline__ void prep_part(const LayerParams& p, const int32_t* seq_len, int max_seq_len,
+                                          const float* q, const AttnWs& ws, int part, int b, int tid,
+                                          double* rope_s, int bar_id) {
+  const int L = seq_len[b];
+  if (L < 1 || L > max_seq_len) return;
+  const int n_pairs = p.d_r / 2;
+  double* rope_g = ws.rope + static_cast<int64_t>(b) * (n_pairs + 1) * 2;
+  for (int i = tid; i < n_pairs; i += kPrepThreads) {
+    double sn, cs;
+    sincos(static_cast<double>(L - 1) * rope_inv_freq(p, i), &sn, &cs);
+    rope_s[2 * i] = cs;
+    rope_s[2 * i + 1] = sn;
+    if (part == 0) {
+      rope_g[2 * i] = cs;
+      rope_g[2 * i + 1] = sn;
+    }
+  }
+  if (!ws.qimage) return;
+  group_sync(bar_id);
+  // tensor-core path (H = 64, D = 512): granule g (8 dims) of head h lands at chunk g/8, row h,
+  // 16-byte slot (g % 8) ^ (h % 8) of the operand image; CTA x builds heads 8x .. 8x+7
+  constexpr int kD = 512, kGr = kD / 8, kChunk = 64 * 128;
+  const float* qb = q + static_cast<int64_t>(b) * 64 * kD;
+  uint8_t* img = ws.qimage + static_cast<int64_t>(b) * kQImageBytes;
+  const int first_rope = (kD - p.d_r) / 2;
+  for (int it0 = part * 8 * kGr; it0 < (part + 1) * 8 * kGr; it0 += 2 * kPrepThreads) {
+    float4 raw[2][2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int it = it0 + u * kPrepThreads + tid;
+      const float4* src = reinterpret_cast<const float4*>(qb + (it >> 6) * kD + 8 * (it & 63));
+      raw[u][0] = __ldg(src);
+      raw[u][1] = __ldg(src + 1);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int it = it0 + u * kPrepThreads + tid;
+      const int h = it >> 6, g = it & 63;
+      float v[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                    raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int pr = 4 * g + k;
+        if (pr >= first_rope) {
+          const double cs = rope_s[2 * (pr - first_rope)], sn = rope_s[2 * (pr - first_rope) + 1];
+          const double x0 = v[2 * k], x1 = v[2 * k + 1];
+          v[2 * k] = static_cast<float>(x0 * cs - x1 * sn);
+          v[2 * k + 1] = static_cast<float>(x0 * sn + x1 * cs);
+        }
+      }
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __half2 hh = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+        w[k] = *reinterpret_cast<uint32_t*>(&hh);
+      }
+      const uint32_t off = static_cast<uint32_t>(g >> 3) * kChunk + h * 128 + (((g & 7) ^ (h & 7)) << 4);
+      *reinterpret_cast<uint4*>(img + off) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+}  // namespace ckv
