@@ -269,6 +269,22 @@ def run_cuda(args, w: S.Workload):
         for e in pair:
             e.record(stream)
     torch.cuda.synchronize()
+    # the step (every layer's calls) as one CUDA graph, replayed once per timed step
+    step_graph, step_launch = None, "eager"
+    launches_per_step = None
+    if not args.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            l0 = ckv.launch_count()
+            with torch.cuda.graph(g):
+                step.run()
+            launches_per_step = ckv.launch_count() - l0
+            g.replay()
+            torch.cuda.synchronize()
+            step_graph, step_launch = g, "one CUDA graph per step"
+        except RuntimeError as exc:   # capture refused: stay eager and say so
+            step_launch = "eager (graph capture failed: %s)" % str(exc).splitlines()[0][:120]
+            torch.cuda.synchronize()
     clocks = ClockSampler(local)
     time.sleep(0.3)
     launches0 = ckv.launch_count()
@@ -276,10 +292,14 @@ def run_cuda(args, w: S.Workload):
     for i in range(args.steps):
         flush_l2()
         ev[i][0].record(stream)
-        step.run()
+        if step_graph is not None:
+            step_graph.replay()
+        else:
+            step.run()
         ev[i][1].record(stream)
     barrier()
-    launches = ckv.launch_count() - launches0
+    launches = (launches_per_step * args.steps if step_graph is not None
+                else ckv.launch_count() - launches0)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = max_over_ranks(sum(step_ms), dev)
 
@@ -389,6 +409,7 @@ def run_cuda(args, w: S.Workload):
             "step": "append decode token + indexer/top-k + attention (+ split combine), per layer",
             "api": ("ckv_decode_step, one call per layer" if args.api == "fused"
                     else "kv_compress_append + sparse_indexer_topk + compressed_window_attention"),
+            "launch": step_launch,
         },
         "hbm": {"step_bytes": step_bytes,
                 "step_GBps": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
