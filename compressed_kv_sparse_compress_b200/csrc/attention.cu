@@ -11,8 +11,9 @@
 // un-normalised partial (running max m, sum l, sum of p*x) per head, and attn_combine merges
 // the splits by log-sum-exp, normalises, and rotates the rotary dims back by -(L-1).
 //
-// This file holds the CUDA-core path (any head count, fp32 accumulation of everything) and the
-// combine. The tensor-core path for H=64 lives in attention_tc.cu and writes the same partials.
+// This file holds the query preparation, the CUDA-core path (any head count, fp32 accumulation of
+// everything, fp32 partials) and the two combines. The tensor-core path for H=64, D=512 lives in
+// attention_tc.cu and writes the same partials as fp16 rows with a power-of-two scale each.
 
 #include "ckv_internal.h"
 #include "query_prep.cuh"
@@ -20,9 +21,6 @@
 
 namespace ckv {
 
-bool attention_tc_supported(const LayerParams& p);
-int attention_tc_tiles_per_split(int batch, int64_t max_keys);
-int attention_tc_tile_keys();
 int attention_tc_keys_per_split(int batch, int64_t max_keys);
 cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,
                                 int max_seq_len, const float* q, const int32_t* idx,

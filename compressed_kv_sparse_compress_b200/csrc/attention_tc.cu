@@ -612,8 +612,6 @@ int attention_tc_tiles_per_split(int batch, int64_t max_keys) {
   return static_cast<int>(t < 8 ? t : 8);
 }
 
-int attention_tc_tile_keys() { return kTile; }
-
 int attention_tc_keys_per_split(int batch, int64_t max_keys) {
   // half tiles (64 keys; the MMAs still run at M = 128 over the staged half) while they fit one
   // wave: twice the CTAs, each staging half the rows
