@@ -642,16 +642,16 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
     }
   }
 
-  // one exclusive block scan of (count above T) << 16 | (count equal to T), both <= kSmallMax
-  uint32_t n_gt = 0, n_eq = 0;
+  // masks of this thread's keys above T and equal to T; one exclusive block scan of
+  // (count above) << 16 | (count equal), both <= kSmallMax
+  uint32_t gt = 0, eq = 0;
 #pragma unroll
   for (int u = 0; u < kSmallPerThread; ++u) {
-    if ((valid >> u) & 1u) {
-      n_gt += (all || key[u] > T) ? 1u : 0u;
-      n_eq += (!all && key[u] == T) ? 1u : 0u;
-    }
+    const bool v = (valid >> u) & 1u;
+    gt |= (v && (all || key[u] > T)) ? (1u << u) : 0u;
+    eq |= (v && !all && key[u] == T) ? (1u << u) : 0u;
   }
-  const uint32_t packed = (n_gt << 16) | n_eq;
+  const uint32_t packed = (static_cast<uint32_t>(__popc(gt)) << 16) | static_cast<uint32_t>(__popc(eq));
   const int lane = tid & 31, w = tid >> 5;
   uint32_t incl = packed;
 #pragma unroll
@@ -665,19 +665,22 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
   const uint32_t excl = below + incl - packed;
-  uint32_t eq_before = excl & 0xffffu;
+  const uint32_t eq_before = excl & 0xffffu;
+  // the equal keys taken here: the first (quota - eq_before) of this thread's, in index order
+  uint32_t take = gt;
+  if (eq) {
+    uint32_t rest = eq;
+    const uint32_t n_take = quota > eq_before ? quota - eq_before : 0u;
+    for (uint32_t i = 0; i < n_take && rest; ++i) rest &= rest - 1;  // drop the lowest n_take
+    take |= eq & ~rest;
+  }
   uint32_t pos = (excl >> 16) + (eq_before < quota ? eq_before : quota);
   int32_t* out = idx + static_cast<int64_t>(b) * top_k;
-#pragma unroll
-  for (int u = 0; u < kSmallPerThread; ++u) {
-    if ((valid >> u) & 1u) {
-      bool take = all || key[u] > T;
-      if (!all && key[u] == T) take = eq_before++ < quota;
-      if (take) {
-        if (pos < static_cast<uint32_t>(top_k)) out[pos] = j0 + u;
-        ++pos;
-      }
-    }
+  while (take) {  // ascending index order
+    const int u = __ffs(take) - 1;
+    take &= take - 1;
+    if (pos < static_cast<uint32_t>(top_k)) out[pos] = j0 + u;
+    ++pos;
   }
   for (int i = k_eff + tid; i < top_k; i += kSmallThreads) out[i] = -1;
   if (tid == 0) cnt[b] = k_eff;
