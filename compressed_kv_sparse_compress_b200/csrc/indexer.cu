@@ -67,6 +67,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMarkChunk = 4 * kThreads;  // scores per mark CTA
 constexpr int kFinishThreads = 1024;
+static_assert(kHistBins == 8 * kThreads && kHistBins == 2 * kFinishThreads, "first-digit bins per thread");
 
 // ---------------------------------------------------------------------------- block scans
 
@@ -348,6 +349,44 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int b
 
 // ---------------------------------------------------------------------------- selection
 
+// Boundary of a block-distributed histogram (thread t owns bins [t * NBL, (t + 1) * NBL), NW warps)
+// for selecting `need` items from the top bin down: returns (bin, items in the bins above it) to
+// every thread. Two barriers.
+template <int NBL, int NW>
+__device__ __forceinline__ uint2 small_boundary(const uint32_t (&c)[NBL], uint32_t need, uint32_t* wsum,
+                                                uint2* bnd) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < NBL; ++i) s += c[i];
+  uint32_t suf = s;  // items in this lane's bins and those of the lanes above it
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += t;
+  }
+  if (lane == 0) wsum[w] = suf;
+  __syncthreads();
+  uint32_t above = (lane > w && lane < NW) ? wsum[lane] : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+  above += suf - s;  // items in all bins above this thread's bins
+  if (above < need && above + s >= need) {
+    uint32_t cum = above;
+#pragma unroll
+    for (int i = NBL - 1; i >= 0; --i) {
+      if (cum + c[i] >= need) {
+        *bnd = make_uint2(static_cast<uint32_t>(threadIdx.x * NBL + i), cum);
+        break;
+      }
+      cum += c[i];
+    }
+  }
+  __syncthreads();
+  return *bnd;
+}
+
+
 // One CTA per 1024 scores of a request: each lane classifies 4 consecutive scores against the
 // boundary bin of the first digit; the bitmap word of 32 scores is assembled from 8 lanes.
 __global__ void __launch_bounds__(kThreads) topk_mark_kernel(const float* scores, int64_t stride,
@@ -375,11 +414,13 @@ __global__ void __launch_bounds__(kThreads) topk_mark_kernel(const float* scores
   // the lane's scores (stride is a multiple of 64 floats, so the float4 is in bounds)
   float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
   if (j < N) v = __ldcg(reinterpret_cast<const float4*>(scores + static_cast<int64_t>(b) * stride + j));
+  // first-digit boundary from the score kernel's histogram, eight bins per thread
   __shared__ uint32_t sh[32];
-  __shared__ uint32_t bnd[2];
-  find_boundary(ws.hist + static_cast<int64_t>(b) * kHistBins, kHistBins, static_cast<uint32_t>(top_k),
-                true, sh, bnd);
-  const uint32_t b1 = bnd[0];
+  __shared__ uint2 bnd;
+  const uint4* hg = reinterpret_cast<const uint4*>(ws.hist + static_cast<int64_t>(b) * kHistBins) + 2 * threadIdx.x;
+  const uint4 ha = __ldcg(hg), hb = __ldcg(hg + 1);
+  const uint32_t c8[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
+  const uint32_t b1 = small_boundary<8, kWarps>(c8, static_cast<uint32_t>(top_k), sh, &bnd).x;
   const float vals[4] = {v.x, v.y, v.z, v.w};
   uint32_t keys[4];
   uint32_t sel = 0, cnd = 0;
@@ -441,6 +482,18 @@ __device__ DigitSel candidate_digit_pass(const uint2* cand, uint32_t m, uint32_t
     atomicAdd(h + ((v >> shift) & (nbins - 1)), 1u);
   }
   __syncthreads();
+  __shared__ uint2 sel;
+  if (!kByIndex && nbins == 2 * kFinishThreads) {  // descending, 2 bins per thread
+    const uint2 hv = reinterpret_cast<const uint2*>(h)[threadIdx.x];
+    const uint32_t c2[2] = {hv.x, hv.y};
+    const uint2 r = small_boundary<2, kFinishThreads / 32>(c2, need, sh, &sel);
+    return DigitSel{r.x, r.y};
+  }
+  if (!kByIndex && nbins == kFinishThreads) {  // descending, 1 bin per thread
+    const uint32_t c1[1] = {h[threadIdx.x]};
+    const uint2 r = small_boundary<1, kFinishThreads / 32>(c1, need, sh, &sel);
+    return DigitSel{r.x, r.y};
+  }
   __shared__ uint32_t out[2];
   find_boundary(h, nbins, need, !kByIndex, sh, out);
   return DigitSel{out[0], out[1]};
@@ -455,16 +508,18 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, 
   __shared__ uint32_t h[kHistBins];
   __shared__ uint2 cand_s[kCandSmem];
   __shared__ uint32_t sh[32];
-  __shared__ uint32_t bnd[2];
+  __shared__ uint2 bnd;
   const int b = blockIdx.x;
   const int64_t N = ws.n_c[b];
   const int64_t k_eff = min(static_cast<int64_t>(top_k), N);
   uint32_t* bm = ws.bitmap + static_cast<int64_t>(b) * (stride / 32);
   if (N > top_k) {
-    find_boundary(ws.hist + static_cast<int64_t>(b) * kHistBins, kHistBins, static_cast<uint32_t>(top_k),
-                  true, sh, bnd);
-    const uint32_t b1 = bnd[0];
-    uint32_t need = static_cast<uint32_t>(k_eff) - bnd[1];
+    // first digit from the score kernel's histogram, two bins per thread
+    const uint2 hv = __ldcg(reinterpret_cast<const uint2*>(ws.hist + static_cast<int64_t>(b) * kHistBins) + threadIdx.x);
+    const uint32_t c1[2] = {hv.x, hv.y};
+    const uint2 r1 = small_boundary<2, kFinishThreads / 32>(c1, static_cast<uint32_t>(top_k), sh, &bnd);
+    const uint32_t b1 = r1.x;
+    uint32_t need = static_cast<uint32_t>(k_eff) - r1.y;
     const uint32_t m = ws.cand_cnt[b];
     const uint2* cand = ws.cand + static_cast<int64_t>(b) * stride;
     if (m <= kCandSmem) {
@@ -476,10 +531,20 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, 
     const DigitSel dA = candidate_digit_pass<false>(cand, m, h, 10, 11, 0xffe00000u, b1 << 21, 0, need, sh);
     need -= dA.before;
     const uint32_t pA = (b1 << 21) | (dA.bin << 10);
-    const DigitSel dB = candidate_digit_pass<false>(cand, m, h, 0, 10, 0xfffffc00u, pA, 0, need, sh);
-    need -= dB.before;
-    const uint32_t T = pA | dB.bin;
-    const uint32_t n_eq = h[dB.bin];
+    uint32_t T, n_eq;
+    if (h[dA.bin] == need) {
+      // every candidate of the boundary bin is taken: select key >= the bin's lower edge pA
+      // (key == pA with any index)
+      T = pA;
+      n_eq = 0;
+      need = 0;
+    } else {
+      __syncthreads();  // every thread has read h before the next pass clears it
+      const DigitSel dB = candidate_digit_pass<false>(cand, m, h, 0, 10, 0xfffffc00u, pA, 0, need, sh);
+      need -= dB.before;
+      T = pA | dB.bin;
+      n_eq = h[dB.bin];
+    }
     // among key == T keep the `need` lowest indices: index threshold by three ascending digits
     uint32_t idx_thr = 0xffffffffu;
     if (need < n_eq) {
@@ -534,42 +599,6 @@ constexpr int kSmallWarps = kSmallThreads / 32;
 constexpr int kSmallPerThread = 32;
 constexpr int kSmallMax = kSmallThreads * kSmallPerThread;
 
-// Boundary of a block-distributed histogram for selecting `need` items from the top bin down:
-// returns (bin, items in the bins above it) to every thread.
-template <int NBL>
-__device__ __forceinline__ uint2 small_boundary(const uint32_t (&c)[NBL], uint32_t need, uint32_t* wsum,
-                                                uint2* bnd) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  uint32_t s = 0;
-#pragma unroll
-  for (int i = 0; i < NBL; ++i) s += c[i];
-  uint32_t suf = s;  // items in this lane's bins and those of the lanes above it
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_down_sync(0xffffffffu, suf, o);
-    if (lane + o < 32) suf += t;
-  }
-  if (lane == 0) wsum[w] = suf;
-  __syncthreads();
-  uint32_t above = (lane > w && lane < kSmallWarps) ? wsum[lane] : 0u;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
-  above += suf - s;  // items in all bins above this thread's bins
-  if (above < need && above + s >= need) {
-    uint32_t cum = above;
-#pragma unroll
-    for (int i = NBL - 1; i >= 0; --i) {
-      if (cum + c[i] >= need) {
-        *bnd = make_uint2(static_cast<uint32_t>(threadIdx.x * NBL + i), cum);
-        break;
-      }
-      cum += c[i];
-    }
-  }
-  __syncthreads();
-  return *bnd;
-}
-
 __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* scores, int64_t stride,
                                                                    int nmax, int top_k, IndexerWs ws,
                                                                    int32_t* idx, int32_t* cnt) {
@@ -613,7 +642,7 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
   uint32_t T = 0, quota = 0;  // selected: key > T, and the first `quota` keys == T in index order
   if (!all) {
     const uint32_t c1[4] = {c1v.x, c1v.y, c1v.z, c1v.w};
-    const uint2 r1 = small_boundary<4>(c1, static_cast<uint32_t>(k_eff), wsum[0], &bnd);
+    const uint2 r1 = small_boundary<4, kSmallWarps>(c1, static_cast<uint32_t>(k_eff), wsum[0], &bnd);
     const uint32_t need2 = static_cast<uint32_t>(k_eff) - r1.y;
 #pragma unroll
     for (int u = 0; u < kSmallPerThread; ++u)
@@ -621,7 +650,7 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
     __syncthreads();
     const uint4 c2v = reinterpret_cast<const uint4*>(h2)[tid];
     const uint32_t c2[4] = {c2v.x, c2v.y, c2v.z, c2v.w};
-    const uint2 r2 = small_boundary<4>(c2, need2, wsum[1], &bnd);
+    const uint2 r2 = small_boundary<4, kSmallWarps>(c2, need2, wsum[1], &bnd);
     const uint32_t need3 = need2 - r2.y;
     const uint32_t p2 = (r1.x << 11) | r2.x;
     if (h2[r2.x] == need3 && p2 > 0) {
@@ -636,7 +665,7 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
       __syncthreads();
       const uint2 c3v = reinterpret_cast<const uint2*>(h3)[tid];
       const uint32_t c3[2] = {c3v.x, c3v.y};
-      const uint2 r3 = small_boundary<2>(c3, need3, wsum[0], &bnd);
+      const uint2 r3 = small_boundary<2, kSmallWarps>(c3, need3, wsum[0], &bnd);
       T = (p2 << 10) | r3.x;
       quota = need3 - r3.y;
     }
