@@ -289,9 +289,10 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u) {
 // (request, group of kGH heads). Each split's partial rows of the group are 4 KB of contiguous
 // memory; up to kGS splits per round are bulk-copied into shared memory while the block reduces
 // their (m, l) per head, and thread t then merges dims 8 (t % 64) .. 8 (t % 64) + 7 of head
-// t / 64 of the group from shared memory (running max and sums rescaled between rounds).
+// t / 64 of the group from shared memory (running max and sums rescaled between rounds). The
+// shared memory holds the rounds' rows: min(splits, kGS) x 4 KB.
 constexpr int kGH = 4;
-constexpr int kGS = 16;
+constexpr int kGS = 48;  // splits per round (48 x 4 KB = 192 KB of shared memory)
 constexpr int kGThreads = 256;
 constexpr int kGDim = 512;
 constexpr uint32_t kGRow = kGH * kGDim * 2;
