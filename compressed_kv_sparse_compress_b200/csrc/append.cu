@@ -503,7 +503,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
 // sparse layers, the query preparation alone on dense ones), which reads only the query. The two
 // halves synchronise on barriers 1 and 2 and never wait for each other.
 template <bool kSparse>
-__global__ void __launch_bounds__(2 * kAppendThreads, kSparse ? 1 : 2) step_front_kernel(
+__global__ void __launch_bounds__(2 * kAppendThreads, 1) step_front_kernel(
     AppendArgs a, int app_slices, const float* q, IndexerWs iws, QueryPrepOut prep, AttnWs aws,
     int prep_parts) {
   griddep_wait();
