@@ -17,11 +17,16 @@ pytestmark = pytest.mark.gpu
 
 CACHE_PLANES = ("comp_codes", "comp_scales", "win_codes", "win_scales", "residue_kv", "residue_logit")
 
+# batches of up to 18 requests launch the append and the query pass as two kernels, larger ones as
+# one front kernel (more (request, slice) CTAs than SMs): both forms are covered
+_LENS24 = tuple(1000 + (7919 * i) % 30000 for i in range(24))
 SMALL = [
     S.scaled(S.csa_b8_ctx32k(), (32768, 20001, 4099, 9, 700, 131), "fused", seed=6000),
     S.scaled(S.hca_b32_ctx128k(), (131072, 60000, 129, 1000), "fused", seed=6001),
     S.scaled(S.mixed_64req(), (16385, 5000, 1025, 70000), "fused", seed=6002),
     S.csa_b1_ctx4k_fp32(),
+    S.scaled(S.csa_b8_ctx32k(), _LENS24, "fused_front", seed=6003),
+    S.scaled(S.hca_b32_ctx128k(), tuple(4 * x for x in _LENS24), "fused_front", seed=6004),
 ]
 
 
