@@ -15,7 +15,7 @@
 //                   non-allocating loads, writes its fp32 score, and counts the top 11 bits of
 //                   its order key into a per-request histogram (first radix digit)
 //   topk_small      per request, when every request has at most 16384 candidates: the whole
-//                   selection in one CTA with the scores in registers
+//                   selection in one CTA of 1024 threads with the scores in registers
 //   topk_mark       per (request, 8192 scores): marks scores above the boundary bin in a
 //                   bitmap and appends boundary-bin candidates to a list
 //   topk_finish     per request: resolves the boundary bin with two more radix digits (and the
@@ -594,9 +594,9 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, 
 // barriers per digit; the first digit's histogram is the one the score kernel counted. Ties at
 // the threshold key go to the lowest indices and the winners are written in ascending order, both
 // from one block scan of the packed pair (count above the threshold, count equal to it).
-constexpr int kSmallThreads = 512;
+constexpr int kSmallThreads = 1024;
 constexpr int kSmallWarps = kSmallThreads / 32;
-constexpr int kSmallPerThread = 32;
+constexpr int kSmallPerThread = 16;
 constexpr int kSmallMax = kSmallThreads * kSmallPerThread;
 
 __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* scores, int64_t stride,
@@ -609,7 +609,7 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
   __shared__ uint32_t wsum[2][kSmallWarps];
   __shared__ uint2 bnd;
   const int b = blockIdx.x, tid = threadIdx.x;
-  const int per = (nmax + 4 * kSmallThreads - 1) / (4 * kSmallThreads) * 4;  // multiple of 4, <= 32
+  const int per = (nmax + 4 * kSmallThreads - 1) / (4 * kSmallThreads) * 4;  // multiple of 4, <= 16
   const int j0 = tid * per;
   const float* sb = scores + static_cast<int64_t>(b) * stride;
 
@@ -619,7 +619,7 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
   for (int v = 0; v < kSmallPerThread / 4; ++v)
     raw[v] = (4 * v < per && j0 + 4 * v < nmax) ? __ldcg(reinterpret_cast<const float4*>(sb + j0) + v)
                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-  const uint4 c1v = __ldcg(reinterpret_cast<const uint4*>(ws.hist + static_cast<int64_t>(b) * kHistBins) + tid);
+  const uint2 c1v = __ldcg(reinterpret_cast<const uint2*>(ws.hist + static_cast<int64_t>(b) * kHistBins) + tid);
   const int N = ws.n_c[b];
   for (int i = tid; i < kHistBins; i += kSmallThreads) h2[i] = 0;
   for (int i = tid; i < kHistBins / 2; i += kSmallThreads) h3[i] = 0;
@@ -641,16 +641,16 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
   const bool all = N <= top_k;
   uint32_t T = 0, quota = 0;  // selected: key > T, and the first `quota` keys == T in index order
   if (!all) {
-    const uint32_t c1[4] = {c1v.x, c1v.y, c1v.z, c1v.w};
-    const uint2 r1 = small_boundary<4, kSmallWarps>(c1, static_cast<uint32_t>(k_eff), wsum[0], &bnd);
+    const uint32_t c1[2] = {c1v.x, c1v.y};
+    const uint2 r1 = small_boundary<2, kSmallWarps>(c1, static_cast<uint32_t>(k_eff), wsum[0], &bnd);
     const uint32_t need2 = static_cast<uint32_t>(k_eff) - r1.y;
 #pragma unroll
     for (int u = 0; u < kSmallPerThread; ++u)
       if (((valid >> u) & 1u) && (key[u] >> 21) == r1.x) atomicAdd(h2 + ((key[u] >> 10) & 2047u), 1u);
     __syncthreads();
-    const uint4 c2v = reinterpret_cast<const uint4*>(h2)[tid];
-    const uint32_t c2[4] = {c2v.x, c2v.y, c2v.z, c2v.w};
-    const uint2 r2 = small_boundary<4, kSmallWarps>(c2, need2, wsum[1], &bnd);
+    const uint2 c2v = reinterpret_cast<const uint2*>(h2)[tid];
+    const uint32_t c2[2] = {c2v.x, c2v.y};
+    const uint2 r2 = small_boundary<2, kSmallWarps>(c2, need2, wsum[1], &bnd);
     const uint32_t need3 = need2 - r2.y;
     const uint32_t p2 = (r1.x << 11) | r2.x;
     if (h2[r2.x] == need3 && p2 > 0) {
@@ -663,9 +663,8 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
       for (int u = 0; u < kSmallPerThread; ++u)
         if (((valid >> u) & 1u) && (key[u] >> 10) == p2) atomicAdd(h3 + (key[u] & 1023u), 1u);
       __syncthreads();
-      const uint2 c3v = reinterpret_cast<const uint2*>(h3)[tid];
-      const uint32_t c3[2] = {c3v.x, c3v.y};
-      const uint2 r3 = small_boundary<2, kSmallWarps>(c3, need3, wsum[0], &bnd);
+      const uint32_t c3[1] = {h3[tid]};
+      const uint2 r3 = small_boundary<1, kSmallWarps>(c3, need3, wsum[0], &bnd);
       T = (p2 << 10) | r3.x;
       quota = need3 - r3.y;
     }
