@@ -533,3 +533,95 @@ def decode_layer(cfg: LayerCfg, cache: LayerCache, b: int, q_raw: np.ndarray, se
         scores = indexer_scores(cfg, cache, b, q_raw, seq_len)
         sel = topk_select(scores, top_k)
     return sel, scores, attention(cfg, cache, b, q_raw, seq_len, sel)
+
+
+# ------------------------------------------------------------------------------------------------
+# Multi-head indexer ([CZ] §C: "Sparse MQA logits" scores only the candidate positions).
+# reading (the second indexer form): the indexer has its own H_I heads of width d_I and its own
+# compressed key per entry. Per token the caller supplies an index key (position encoding, if
+# any, already applied: the projections that make index keys and queries lie outside this path);
+# the index keys of a group are folded with the same softmax weights of the same logits as the
+# K=V tokens ([HR] §A) and stored as FP8 with one fp32 scale per entry (the window's FP8 rule).
+# The decode step supplies one index query per head and one weight per head; the score of
+# candidate j is s_j = sum_h w_h * max(0, q^_h . k_j), where q^ is the index query rounded to
+# fp16 (the precision the scoring takes it in) and k_j the decoded entry. No softmax scale (the
+# weights carry it); top-k as for the head-averaged score.
+# ------------------------------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class IndexCfg:
+    """index_heads: H_I; index_dim: d_I (index key and query width)."""
+    index_heads: int
+    index_dim: int
+
+
+@dataclass
+class IndexCache:
+    """The index-key plane of a layer's compressed pool (same blocks, rows and table).
+
+    codes: uint8 [comp_blocks, 256/r, d_I] e4m3; scales: float32 [comp_blocks, 256/r];
+    residue: per request, the index keys of the unfinished group as (position, key f32 [d_I],
+    logit f32)."""
+    codes: np.ndarray
+    scales: np.ndarray
+    residue: list = field(default_factory=list)
+
+
+def index_append_tokens(cfg: LayerCfg, icache: IndexCache, comp_table: np.ndarray, b: int,
+                        prev_len: int, k_new: np.ndarray, logit_new: np.ndarray) -> None:
+    """Append n index keys (positions prev_len .. prev_len+n-1) of request b; a key that
+    completes a group folds the group (compress_group, no rotation) into entry (pos+1)/r - 1,
+    stored with quantize_fp8_token."""
+    d_i = icache.codes.shape[-1]
+    k_new = np.asarray(k_new, dtype=np.float32).reshape(-1, d_i)
+    logit_new = np.asarray(logit_new, dtype=np.float32).reshape(-1)
+    while len(icache.residue) <= b:
+        icache.residue.append([])
+    res = icache.residue[b]
+    if len(res) != prev_len % cfg.ratio:
+        raise ValueError("index residue does not match prev_len")
+    flat_c = icache.codes.reshape(-1, d_i)
+    flat_s = icache.scales.reshape(-1)
+    for t in range(k_new.shape[0]):
+        pos = prev_len + t
+        res.append((pos, k_new[t].copy(), np.float32(logit_new[t])))
+        if (pos + 1) % cfg.ratio == 0:
+            keys = np.stack([k for _, k, _ in res]).astype(np.float64)
+            lg = np.array([l for _, _, l in res], dtype=np.float64)
+            c = compress_group(keys, lg)
+            row = int(comp_entry_rows(comp_table[b], [(pos + 1) // cfg.ratio - 1], cfg.ratio)[0])
+            codes, s = quantize_fp8_token(c.astype(np.float32))
+            flat_c[row] = codes
+            flat_s[row] = s
+            res.clear()
+
+
+def decode_index_entries(cfg: LayerCfg, icache: IndexCache, comp_table: np.ndarray, b: int,
+                         entries) -> np.ndarray:
+    """fp64 index keys [n, d_I] of the given entries of request b."""
+    rows = comp_entry_rows(comp_table[b], entries, cfg.ratio)
+    d_i = icache.codes.shape[-1]
+    return dequant_fp8_token(icache.codes.reshape(-1, d_i)[rows], 1.0) * \
+        icache.scales.reshape(-1)[rows].astype(np.float64)[:, None]
+
+
+def index_query_f16(q_index: np.ndarray) -> np.ndarray:
+    """The index query as scored: each fp32 element rounded to the nearest fp16 (ties to even)."""
+    return np.asarray(q_index, dtype=np.float32).astype(np.float16).astype(np.float64)
+
+
+def mh_indexer_scores(cfg: LayerCfg, icache: IndexCache, comp_table: np.ndarray, b: int,
+                      q_index: np.ndarray, weights: np.ndarray, seq_len: int,
+                      chunk: int = 16384) -> np.ndarray:
+    """fp64 scores s_j = sum_h w_h max(0, q^_h . k_j) for j < floor(L/r).
+
+    q_index: [H_I, d_I] fp32; weights: [H_I] fp32."""
+    n_c = num_compressed(seq_len, cfg.ratio)
+    qh = index_query_f16(q_index)
+    w = np.asarray(weights, dtype=np.float32).astype(np.float64)
+    out = np.empty(n_c, dtype=np.float64)
+    for j0 in range(0, n_c, chunk):
+        j1 = min(n_c, j0 + chunk)
+        k = decode_index_entries(cfg, icache, comp_table, b, np.arange(j0, j1))
+        out[j0:j1] = np.maximum(k @ qh.T, 0.0) @ w
+    return out

@@ -13,6 +13,10 @@ Recipe (the same for every workload):
     110*N(0,1) clamped to +-440 with an fp32 scale uniform in [0.8, 1.2]/110.
   * block tables: a seeded random permutation of the pool's block ids, dealt to the requests in
     order (``paged``), or the identity (contiguous cache). Unmapped logical blocks are -1.
+  * multi-head indexer (CSA layers, 64 index heads x 128 dims unless stated): index query
+    N(0,1) fp32 [B, H_I, d_I]; head weights N(0,1)/sqrt(H_I) fp32 [B, H_I]; stored index entries
+    FP8 like the window (e4m3 of 110*N(0,1) clamped to +-440, scale uniform in [0.8, 1.2]/110);
+    index keys appended through the compressor N(0,1) fp32 (their logits are the layer's).
   * context lengths of the mixed workload: round(LogNormal(ln 16384, 1.0)) clipped to
     [1024, 524288] for the tokens already cached, plus the decode token.
 
@@ -266,4 +270,26 @@ def generate(w: Workload, device="cpu") -> dict:
         lay["kv_new"] = _randn((B, D), g(8), device)
         lay["logit_new"] = _randn((B,), g(9), device)
         out["layers"].append(lay)
+    return out
+
+
+def generate_index(w: Workload, gen: dict, layer: int = 0, heads: int = 64, dim: int = 128,
+                   device="cpu") -> dict:
+    """Inputs of the multi-head indexer for layer ``layer`` of workload w, whose other inputs
+    ``gen`` holds (the index plane shares that layer's compressed blocks and table).
+
+    Returns: q_index f32 [B, H_I, d_I]; weights f32 [B, H_I]; codes uint8 [blocks, 256/r, d_I];
+    scales f32 [blocks, 256/r]; k_setup f32 [sum, d_I] and k_new f32 [B, d_I] (the index keys of
+    the tokens the layer appends before and at the step)."""
+    lay = gen["layers"][layer]
+    B = w.batch
+    n_blocks, epb = lay["comp_codes"].shape[0], lay["comp_codes"].shape[1]
+    g = lambda s: _gen(device, w.seed, 100 * layer + 20 + s)  # noqa: E731
+    out = {"q_index": _randn((B, heads, dim), g(1), device),
+           "weights": _randn((B, heads), g(2), device) / math.sqrt(heads)}
+    codes, scales = _random_win_pool("fp8", n_blocks * epb, dim, g(3), device)
+    out["codes"] = codes.view(n_blocks, epb, dim)
+    out["scales"] = scales.view(n_blocks, epb)
+    out["k_setup"] = _randn((lay["kv_setup"].shape[0], dim), g(4), device)
+    out["k_new"] = _randn((B, dim), g(5), device)
     return out
