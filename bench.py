@@ -56,16 +56,25 @@ def token_bytes(ls: S.LayerSpec, d: int) -> int:
     return S.win_code_bytes(ls.win_dtype, d) + (4 if ls.win_dtype == "fp8" else 0)
 
 
-def layer_bytes(w: S.Workload, ls: S.LayerSpec) -> dict:
-    """Bytes a step must move for one layer: the indexer reads every candidate once; attention
-    reads the selected entries, the window tokens, the query and writes the output; the append
-    reads the unfinished group's ring and writes one entry and one window token."""
+MH_HEADS, MH_DIM = 64, 128  # multi-head indexer: index heads x index dim
+
+
+def layer_bytes(w: S.Workload, ls: S.LayerSpec, indexer: str = "avg") -> dict:
+    """Bytes a step must move for one layer: the indexer reads every candidate once (its K=V
+    entry for the head-averaged score; its FP8 index entry and scale for the multi-head score);
+    attention reads the selected entries, the window tokens, the query and writes the output; the
+    append reads the unfinished group's ring and writes one entry and one window token (the
+    multi-head form also appends the index key: its ring, one FP8 entry)."""
     d, h = w.head_dim, w.num_heads
     idx_b = att_b = app_b = 0
     for L in w.seq_lens:
         n_c = L // ls.ratio
         if ls.top_k is not None:
-            idx_b += n_c * entry_bytes(ls, d) + 4 * math.ceil(L / 256) + 4 * h * d
+            if indexer == "mh":
+                idx_b += n_c * (MH_DIM + 4) + 4 * math.ceil(L / 256) + 4 * MH_HEADS * (MH_DIM + 1)
+                app_b += 4 * MH_DIM + 4 + (ls.ratio - 1) * (4 * MH_DIM + 4) + MH_DIM + 4
+            else:
+                idx_b += n_c * entry_bytes(ls, d) + 4 * math.ceil(L / 256) + 4 * h * d
             sel = min(ls.top_k, n_c)
         else:
             sel = n_c
@@ -97,6 +106,21 @@ def max_over_ranks(x: float, device="cpu") -> float:
 def job_throughput(units_per_rank_step: int, world: int, steps: int, max_total_ms: float) -> float:
     """Whole-job rate: the units every rank processed in `steps` steps over the slowest rank's time."""
     return units_per_rank_step * world * steps / (max_total_ms / 1e3)
+
+
+def tensor_record(w: S.Workload, indexer: str, avg_ms: float) -> dict:
+    """Tensor-core side of the multi-head score kernel: 2 H_I d_I flops per candidate (fp16
+    operands), against the measured dense bf16 rate (fp16 runs at the same rate)."""
+    n_c = sum(L // ls.ratio for ls in w.layers if ls.top_k is not None for L in w.seq_lens)
+    flops = 2.0 * MH_HEADS * MH_DIM * n_c
+    try:
+        with open(PEAKS_FILE) as f:
+            peak, src = float(json.load(f)["bf16_tflops"]), "measured bf16 burst"
+    except Exception:
+        peak, src = 1590.0, "fallback"
+    ach = flops / (avg_ms / 1e3) / 1e12
+    return {"flops_per_launch": flops, "achieved_tflops": ach, "peak_tflops": peak, "peak_source": src,
+            "frac": ach / peak}
 
 
 def measured_peak():
@@ -178,15 +202,16 @@ def traffic_record(kernel: str, workload: str):
 class Step:
     """All layers of a workload on one GPU, with the step's inputs resident in HBM."""
 
-    def __init__(self, ckv, w: S.Workload, seed_offset: int = 0, api: str = "fused"):
-        self.ckv, self.w, self.api = ckv, w, api
+    def __init__(self, ckv, w: S.Workload, seed_offset: int = 0, api: str = "fused", indexer: str = "avg"):
+        self.ckv, self.w, self.api, self.indexer = ckv, w, api, indexer
         wseed = S.Workload(w.name, w.seq_lens, w.num_heads, w.head_dim, w.rope_dim, w.window,
                            w.layers, w.paged, w.from_scratch, w.seed + seed_offset, w.description)
         self.gen = S.generate(wseed, "cuda")
         self.seq = self.gen["seq_len"]
         self.prev = (self.seq - 1).to(torch.int32)
         self.layers = []
-        for lay, ls in zip(self.gen["layers"], w.layers):
+        self.index = []  # per layer: None, or the multi-head indexer's plane, inputs and workspace
+        for li, (lay, ls) in enumerate(zip(self.gen["layers"], w.layers)):
             cfg = ckv.LayerConfig(w.num_heads, w.head_dim, w.rope_dim, ls.ratio, w.window,
                                   ls.comp_dtype, ls.win_dtype)
             cache = ckv.cache_from_tensors(cfg, w.batch, lay["comp_codes"], lay["comp_scales"],
@@ -198,22 +223,51 @@ class Step:
             if n > 0:  # the unfinished group before the decode token (setup, untimed)
                 dl.append(lay["setup_start"].to(torch.int32), lay["kv_setup"], lay["logit_setup"],
                           cu_new=cu, max_new=n)
+            mh = None
+            if indexer == "mh" and ls.top_k is not None:
+                ix = S.generate_index(wseed, self.gen, layer=li, heads=MH_HEADS, dim=MH_DIM, device="cuda")
+                icfg = ckv.IndexConfig(MH_HEADS, MH_DIM)
+                icache = ckv.IndexCache(ix["codes"], ix["scales"],
+                                        torch.zeros((w.batch, ls.ratio, MH_DIM), device="cuda"),
+                                        torch.zeros((w.batch, ls.ratio), device="cuda"))
+                if n > 0:
+                    ckv.kv_index_append(cfg, cache, icfg, icache, lay["setup_start"].to(torch.int32),
+                                        ix["k_setup"], lay["logit_setup"], dl.status, cu_new=cu, max_new=n,
+                                        max_seq_len=dl.max_seq_len)
+                wsb = ckv.mh_indexer_workspace_bytes(cfg, icfg, w.batch, dl.max_seq_len, ls.top_k)
+                mh = {"ix": ix, "icfg": icfg, "icache": icache,
+                      "ws": torch.empty(wsb, dtype=torch.uint8, device="cuda")}
             self.layers.append((dl, lay))
+            self.index.append(mh)
         torch.cuda.synchronize()
 
-    def run(self, q_list=None, kv_list=None, lg_list=None, seq=None, prev=None):
+    def inputs(self, i):
+        """The step's inputs of layer i: q, new token, its logit, and (multi-head) the index
+        query, head weights and new index key."""
+        lay, mh = self.layers[i][1], self.index[i]
+        extra = [] if mh is None else [mh["ix"]["q_index"], mh["ix"]["weights"], mh["ix"]["k_new"]]
+        return [lay["q"], lay["kv_new"], lay["logit_new"]] + extra
+
+    def run_layer(self, i, seq, prev, ins):
+        dl, mh = self.layers[i][0], self.index[i]
+        q, kv, lg = ins[:3]
+        if mh is not None:
+            qi, wt, kn = ins[3:]
+            dl.append(prev, kv, lg)
+            self.ckv.kv_index_append(dl.cfg, dl.cache, mh["icfg"], mh["icache"], prev, kn, lg, dl.status,
+                                     max_seq_len=dl.max_seq_len)
+            self.ckv.sparse_mh_indexer_topk(dl.cfg, dl.cache, mh["icfg"], mh["icache"], seq, dl.max_seq_len, qi,
+                                            wt, dl.top_k, dl.idx, dl.cnt, mh["ws"], dl.status)
+            return dl.attend(seq, q)
+        if self.api == "fused":
+            return dl.fused_step(seq, q, kv, lg)
+        return dl.step(seq, prev, q, kv, lg)
+
+    def run(self, ins_list=None, seq=None, prev=None):
         seq = self.seq if seq is None else seq
         prev = self.prev if prev is None else prev
-        outs = []
-        for i, (dl, lay) in enumerate(self.layers):
-            q = lay["q"] if q_list is None else q_list[i]
-            kv = lay["kv_new"] if kv_list is None else kv_list[i]
-            lg = lay["logit_new"] if lg_list is None else lg_list[i]
-            if self.api == "fused":
-                outs.append(dl.fused_step(seq, q, kv, lg))
-            else:
-                outs.append(dl.step(seq, prev, q, kv, lg))
-        return outs
+        return [self.run_layer(i, seq, prev, self.inputs(i) if ins_list is None else ins_list[i])
+                for i in range(len(self.layers))]
 
     def status(self) -> int:
         return max(int(dl.status[0].item()) & 0xffffffff for dl, _ in self.layers)
@@ -229,7 +283,7 @@ def run_cuda(args, w: S.Workload):
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
-    step = Step(ckv, w, seed_offset=rank, api=args.api)
+    step = Step(ckv, w, seed_offset=rank, api=args.api, indexer=args.indexer)
     flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_sink = torch.empty(1, dtype=torch.float32, device=dev)
@@ -245,9 +299,10 @@ def run_cuda(args, w: S.Workload):
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
-    dominant = "score_kernel" if any(ls.top_k is not None for ls in w.layers) else "attention_kernel"
-    prof_which = ckv.CKV_PROF_SCORE if dominant == "score_kernel" else ckv.CKV_PROF_ATTENTION
-    n_dom = sum(1 for ls in w.layers if (ls.top_k is not None) == (dominant == "score_kernel"))
+    sparse = any(ls.top_k is not None for ls in w.layers)
+    dominant = "attention_kernel" if not sparse else ("mh_score_kernel" if args.indexer == "mh" else "score_kernel")
+    prof_which = ckv.CKV_PROF_ATTENTION if dominant == "attention_kernel" else ckv.CKV_PROF_SCORE
+    n_dom = sum(1 for ls in w.layers if (ls.top_k is not None) == (dominant != "attention_kernel"))
 
     for _ in range(args.warmup):
         flush_l2()
@@ -312,17 +367,14 @@ def run_cuda(args, w: S.Workload):
             step.run()
         else:  # one event pair per layer of the dominant kind
             k = 0
-            for dl, lay in step.layers:
-                is_dom = (dl.top_k is not None) == (dominant == "score_kernel")
+            for li, (dl, lay) in enumerate(step.layers):
+                is_dom = (dl.top_k is not None) == (dominant != "attention_kernel")
                 if is_dom:
                     ckv.profile_events(prof_which, kev[i][k][0], kev[i][k][1])
                     k += 1
                 else:
                     ckv.profile_events(prof_which)
-                if args.api == "fused":
-                    dl.fused_step(step.seq, lay["q"], lay["kv_new"], lay["logit_new"])
-                else:
-                    dl.step(step.seq, step.prev, lay["q"], lay["kv_new"], lay["logit_new"])
+                step.run_layer(li, step.seq, step.prev, step.inputs(li))
         kstep[i][1].record(stream)
     barrier()
     ckv.profile_events(prof_which)
@@ -333,24 +385,22 @@ def run_cuda(args, w: S.Workload):
         raise RuntimeError(f"device status {step.status():#x} in the timed region")
 
     # ---- end to end through the public API: pinned host inputs -> device -> result on host
-    q_h = [lay["q"].cpu().pin_memory() for _, lay in step.layers]
-    kv_h = [lay["kv_new"].cpu().pin_memory() for _, lay in step.layers]
-    lg_h = [lay["logit_new"].cpu().pin_memory() for _, lay in step.layers]
+    ins_h = [[x.cpu().pin_memory() for x in step.inputs(i)] for i in range(len(step.layers))]
     seq_h = step.seq.cpu().pin_memory()
     out_h = [torch.empty_like(lay["q"], device="cpu").pin_memory() for _, lay in step.layers]
-    q_d = [torch.empty_like(x, device=dev) for x in q_h]
-    kv_d = [torch.empty_like(x, device=dev) for x in kv_h]
-    lg_d = [torch.empty_like(x, device=dev) for x in lg_h]
+    ins_d = [[torch.empty_like(x, device=dev) for x in row] for row in ins_h]
     seq_d = torch.empty_like(seq_h, device=dev)
-    h2d = sum(x.numel() * x.element_size() for x in q_h + kv_h + lg_h) + seq_h.numel() * 4
+    h2d = sum(x.numel() * x.element_size() for row in ins_h for x in row) + seq_h.numel() * 4
     d2h = sum(x.numel() * x.element_size() for x in out_h)
+    need_prev = step.api == "calls" or args.indexer == "mh"
 
     def e2e_step():
         seq_d.copy_(seq_h, non_blocking=True)
-        for a, b in zip(q_d + kv_d + lg_d, q_h + kv_h + lg_h):
-            a.copy_(b, non_blocking=True)
-        prev_d = (seq_d - 1).to(torch.int32) if step.api == "calls" else None
-        outs = step.run(q_d, kv_d, lg_d, seq_d, prev_d)
+        for row_d, row_h in zip(ins_d, ins_h):
+            for a, b in zip(row_d, row_h):
+                a.copy_(b, non_blocking=True)
+        prev_d = (seq_d - 1).to(torch.int32) if need_prev else None
+        outs = step.run(ins_d, seq_d, prev_d)
         for o, oh in zip(outs, out_h):
             oh.copy_(o, non_blocking=True)
 
@@ -385,8 +435,8 @@ def run_cuda(args, w: S.Workload):
     units = w.batch * len(w.layers) * ws  # queries*layers per step over all ranks
     value = job_throughput(w.batch * len(w.layers), ws, args.steps, total_ms)
     peak, peak_src = measured_peak()
-    lb = [layer_bytes(w, ls) for ls in w.layers]
-    if dominant == "score_kernel":
+    lb = [layer_bytes(w, ls, args.indexer) for ls in w.layers]
+    if dominant != "attention_kernel":
         dom_bytes = sum(b["indexer"] for b, ls in zip(lb, w.layers) if ls.top_k is not None) / n_dom
     else:
         dom_bytes = sum(b["attention"] for b, ls in zip(lb, w.layers) if ls.top_k is None) / n_dom
@@ -407,8 +457,12 @@ def run_cuda(args, w: S.Workload):
             "l2": "flushed before every step outside the step events: 256 MiB written, then another "
                   "256 MiB read (the written lines are evicted before the step)",
             "step": "append decode token + indexer/top-k + attention (+ split combine), per layer",
-            "api": ("ckv_decode_step, one call per layer" if args.api == "fused"
+            "api": ("kv_compress_append + kv_index_append + sparse_mh_indexer_topk + "
+                    "compressed_window_attention on sparse layers" if args.indexer == "mh"
+                    else "ckv_decode_step, one call per layer" if args.api == "fused"
                     else "kv_compress_append + sparse_indexer_topk + compressed_window_attention"),
+            "indexer": (f"multi-head: {MH_HEADS} index heads x {MH_DIM} dims, FP8 index entries, fp16 query"
+                        if args.indexer == "mh" else "head-averaged MQA logits over the K=V entries"),
             "launch": step_launch,
         },
         "hbm": {"step_bytes": step_bytes,
@@ -422,6 +476,7 @@ def run_cuda(args, w: S.Workload):
                      "timed_in": "a second pass of K steps with an event pair around every launch "
                                  "of the kernel (that pass: %.1f us per step)" % (kstep_ms / args.steps * 1e3),
                      "traffic": traffic_record(dominant, w.name)},
+        "tensor": tensor_record(w, args.indexer, dom_avg_ms) if dominant == "mh_score_kernel" else None,
         "e2e": {"value": job_throughput(w.batch * len(w.layers), ws, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "launch": graph_note,
                 "ms_per_step": e2e_ms / args.steps},
@@ -457,8 +512,9 @@ def oracle_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_request(w, gen_host, li, b, O):
-    """The oracle's whole step for request b of layer li (append + select + attention)."""
+def oracle_request(w, gen_host, li, b, O, ix_host=None):
+    """The oracle's whole step for request b of layer li (append + select + attention); with
+    ix_host (the multi-head indexer's inputs of that layer) the selection is the multi-head one."""
     ls = w.layers[li]
     lay = gen_host["layers"][li]
     cfg = O.LayerCfg(w.num_heads, w.head_dim, w.rope_dim, ls.ratio, w.window, ls.comp_dtype,
@@ -470,7 +526,16 @@ def oracle_request(w, gen_host, li, b, O):
     cu = lay["cu_setup"]
     O.append_tokens(cfg, cache, b, start, lay["kv_setup"][cu[b]:cu[b + 1]], lay["logit_setup"][cu[b]:cu[b + 1]])
     O.append_tokens(cfg, cache, b, L - 1, lay["kv_new"][b:b + 1], lay["logit_new"][b:b + 1])
-    O.decode_layer(cfg, cache, b, lay["q"][b], L, ls.top_k)
+    if ix_host is None or ls.top_k is None:
+        O.decode_layer(cfg, cache, b, lay["q"][b], L, ls.top_k)
+        return
+    ic = O.IndexCache(ix_host["codes"], ix_host["scales"], residue=[[] for _ in range(w.batch)])
+    O.index_append_tokens(cfg, ic, lay["comp_table"], b, start, ix_host["k_setup"][cu[b]:cu[b + 1]],
+                          lay["logit_setup"][cu[b]:cu[b + 1]])
+    O.index_append_tokens(cfg, ic, lay["comp_table"], b, L - 1, ix_host["k_new"][b:b + 1],
+                          lay["logit_new"][b:b + 1])
+    s = O.mh_indexer_scores(cfg, ic, lay["comp_table"], b, ix_host["q_index"][b], ix_host["weights"][b], L)
+    O.attention(cfg, cache, b, lay["q"][b], L, O.topk_select(s, ls.top_k))
 
 
 def host_inputs(gen):
@@ -481,16 +546,21 @@ def host_inputs(gen):
     return out
 
 
+def index_host(ix):
+    return None if ix is None else {k: v.cpu().numpy().copy() for k, v in ix.items()}
+
+
 def cpu_baseline(w, step, seconds):
     from oracle import ckv_oracle as O
     gen_host = host_inputs(step.gen)
+    ix_host = [index_host(None if mh is None else mh["ix"]) for mh in step.index]
     done = 0
     t0 = time.perf_counter()
     reqs = []
     while True:
         for li in range(len(w.layers)):
             b = done % w.batch
-            oracle_request(w, gen_host, li, b, O)
+            oracle_request(w, gen_host, li, b, O, ix_host[li])
             reqs.append((li, b))
         done += 1
         if time.perf_counter() - t0 >= seconds or done >= 64 * w.batch:
@@ -499,7 +569,8 @@ def cpu_baseline(w, step, seconds):
     return {"value": done * len(w.layers) / el, "unit": UNIT, "cores": oracle_threads(),
             "kind": "oracle",
             "sample": f"{done} requests x {len(w.layers)} layer(s) of {w.name} (same seeded inputs), "
-                      f"each a full append+select+attend in the fp64 numpy oracle; {el:.1f} s"}
+                      f"each a full append+select+attend in the fp64 numpy oracle"
+                      f"{' with the multi-head indexer' if step.indexer == 'mh' else ''}; {el:.1f} s"}
 
 
 def run_reference(args, w):
@@ -509,17 +580,19 @@ def run_reference(args, w):
     from oracle import ckv_oracle as O
     gen = S.generate(w, "cpu")
     gen_host = host_inputs(gen)
+    ix_host = [index_host(S.generate_index(w, gen, layer=li, heads=MH_HEADS, dim=MH_DIM, device="cpu"))
+               if args.indexer == "mh" and ls.top_k is not None else None for li, ls in enumerate(w.layers)]
     per_step = w.batch if args.reference_requests <= 0 else min(w.batch, args.reference_requests)
     b = 0
     for _ in range(args.warmup):
         for li in range(len(w.layers)):
-            oracle_request(w, gen_host, li, b % w.batch, O)
+            oracle_request(w, gen_host, li, b % w.batch, O, ix_host[li])
         b += 1
     t0 = time.perf_counter()
     for _ in range(args.steps):
         for _r in range(per_step):
             for li in range(len(w.layers)):
-                oracle_request(w, gen_host, li, b % w.batch, O)
+                oracle_request(w, gen_host, li, b % w.batch, O, ix_host[li])
             b += 1
     el = time.perf_counter() - t0
     units = args.steps * per_step * len(w.layers)
@@ -529,7 +602,7 @@ def run_reference(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "sample_requests_per_step": per_step,
+        "config": {"workload": w.name, "sample_requests_per_step": per_step, "indexer": args.indexer,
                    "note": "CPU oracle (fp64 numpy) on a bounded sample of the workload's requests"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
                          "sample": f"{per_step} request(s) x {len(w.layers)} layer(s) per step"},
@@ -546,6 +619,9 @@ def main():
     ap.add_argument("--impl", default="ckv", choices=["ckv", "reference"])
     ap.add_argument("--api", default="fused", choices=["fused", "calls"],
                     help="fused: one ckv_decode_step per layer; calls: append, select, attend")
+    ap.add_argument("--indexer", default="avg", choices=["avg", "mh"],
+                    help="avg: head-averaged indexer over the K=V entries; mh: multi-head indexer "
+                         f"({MH_HEADS} heads x {MH_DIM} dims) over its own FP8 index entries")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="end-to-end steps launched eagerly")

@@ -38,7 +38,7 @@ EXPORTS = (
     "ckv_indexer_workspace_bytes", "ckv_attention_workspace_bytes", "kv_compress_append",
     "sparse_indexer_topk", "compressed_window_attention", "ckv_status_str", "ckv_launch_count",
     "ckv_profile_events", "sparse_indexer_topk_noalloc", "ckv_decode_step_workspace_bytes",
-    "ckv_decode_step",
+    "ckv_decode_step", "kv_index_append", "ckv_mh_indexer_workspace_bytes", "sparse_mh_indexer_topk",
 )
 CKV_PROF_SCORE, CKV_PROF_ATTENTION = 0, 1
 
@@ -64,6 +64,15 @@ class LayerCacheC(ctypes.Structure):
                 ("comp_table", ctypes.c_void_p), ("win_table", ctypes.c_void_p),
                 ("table_stride", ctypes.c_int32), ("comp_blocks", ctypes.c_int32),
                 ("win_blocks", ctypes.c_int32)]
+
+
+class IndexCfgC(ctypes.Structure):
+    _fields_ = [("index_heads", ctypes.c_int32), ("index_dim", ctypes.c_int32)]
+
+
+class IndexCacheC(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("residue_k", ctypes.c_void_p), ("residue_logit", ctypes.c_void_p)]
 
 
 _lib = None
@@ -107,6 +116,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ckv_decode_step.argtypes = [P(LayerCfgC), P(LayerCacheC), i32, vp, i32, vp, vp, vp, i32, vp,
                                     vp, vp, vp, sz, vp, vp]
     lib.ckv_decode_step.restype = ctypes.c_int
+    lib.kv_index_append.argtypes = [P(LayerCfgC), P(LayerCacheC), P(IndexCfgC), P(IndexCacheC), i32, vp,
+                                    vp, i32, i32, vp, vp, vp, vp]
+    lib.kv_index_append.restype = ctypes.c_int
+    lib.ckv_mh_indexer_workspace_bytes.argtypes = [P(LayerCfgC), P(IndexCfgC), i32, i32, i32]
+    lib.ckv_mh_indexer_workspace_bytes.restype = sz
+    lib.sparse_mh_indexer_topk.argtypes = [P(LayerCfgC), P(LayerCacheC), P(IndexCfgC), P(IndexCacheC), i32,
+                                           vp, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp, vp]
+    lib.sparse_mh_indexer_topk.restype = ctypes.c_int
     lib.ckv_status_str.argtypes = [ctypes.c_int]
     lib.ckv_status_str.restype = ctypes.c_char_p
     lib.ckv_profile_events.argtypes = [ctypes.c_int, vp, vp]
@@ -325,3 +342,60 @@ def decode_step(cfg: LayerConfig, cache: LayerCache, seq_len: torch.Tensor, max_
         ctypes.byref(cfg.c()), ctypes.byref(cache.c()), batch, _ptr(seq_len), max_seq_len, _ptr(q),
         _ptr(kv_new), _ptr(logit_new), top_k, _ptr(idx), _ptr(cnt), _ptr(out), _ptr(workspace),
         workspace.numel(), _ptr(status), _stream(stream)))
+
+
+# ------------------------------------------------------------------------------ multi-head indexer
+
+
+@dataclass
+class IndexConfig:
+    index_heads: int = 64
+    index_dim: int = 128
+
+    def c(self) -> IndexCfgC:
+        return IndexCfgC(self.index_heads, self.index_dim)
+
+
+@dataclass
+class IndexCache:
+    """Device tensors of a layer's index plane (see ckv_index_cache); the rings may be None for
+    scoring only."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    residue_k: torch.Tensor | None = None
+    residue_logit: torch.Tensor | None = None
+
+    def c(self) -> IndexCacheC:
+        return IndexCacheC(_ptr(self.codes), _ptr(self.scales), _ptr(self.residue_k),
+                           _ptr(self.residue_logit))
+
+
+def kv_index_append(cfg: LayerConfig, cache: LayerCache, icfg: IndexConfig, icache: IndexCache,
+                    prev_len: torch.Tensor, k_new: torch.Tensor, logit_new: torch.Tensor,
+                    status: torch.Tensor, cu_new: torch.Tensor | None = None, max_new: int = 1,
+                    max_seq_len: int | None = None, stream=None) -> None:
+    batch = int(prev_len.shape[0])
+    if max_seq_len is None:
+        max_seq_len = int(cache.comp_table.shape[1]) * 256
+    _check("kv_index_append", load_library().kv_index_append(
+        ctypes.byref(cfg.c()), ctypes.byref(cache.c()), ctypes.byref(icfg.c()), ctypes.byref(icache.c()),
+        batch, _ptr(prev_len), _ptr(cu_new), max_new if cu_new is not None else 1, max_seq_len, _ptr(k_new),
+        _ptr(logit_new), _ptr(status), _stream(stream)))
+
+
+def mh_indexer_workspace_bytes(cfg: LayerConfig, icfg: IndexConfig, batch: int, max_seq_len: int,
+                               top_k: int) -> int:
+    return int(load_library().ckv_mh_indexer_workspace_bytes(ctypes.byref(cfg.c()), ctypes.byref(icfg.c()),
+                                                             batch, max_seq_len, top_k))
+
+
+def sparse_mh_indexer_topk(cfg: LayerConfig, cache: LayerCache, icfg: IndexConfig, icache: IndexCache,
+                           seq_len: torch.Tensor, max_seq_len: int, q_index: torch.Tensor,
+                           weights: torch.Tensor, top_k: int, idx: torch.Tensor, cnt: torch.Tensor,
+                           workspace: torch.Tensor, status: torch.Tensor,
+                           scores: torch.Tensor | None = None, stream=None) -> None:
+    batch = int(seq_len.shape[0])
+    _check("sparse_mh_indexer_topk", load_library().sparse_mh_indexer_topk(
+        ctypes.byref(cfg.c()), ctypes.byref(cache.c()), ctypes.byref(icfg.c()), ctypes.byref(icache.c()),
+        batch, _ptr(seq_len), max_seq_len, _ptr(q_index), _ptr(weights), top_k, _ptr(idx), _ptr(cnt),
+        _ptr(scores), _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)))

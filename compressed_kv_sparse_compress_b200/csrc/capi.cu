@@ -150,6 +150,36 @@ int make_params(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int batc
   return CKV_OK;
 }
 
+// Validates the index config and plane. need_residue: the append path.
+int make_index_params(const ckv_index_cfg* icfg, const ckv_index_cache* icache, bool need_residue,
+                      IndexParams* ip) {
+  if (!icfg || !icache) return CKV_ERR_INVALID_ARG;
+  const int H = icfg->index_heads, d = icfg->index_dim;
+  if (H < 16 || H > 128 || H % 16 != 0) return CKV_ERR_UNSUPPORTED;
+  if (d != 128 && d != 256) return CKV_ERR_UNSUPPORTED;
+  if (!icache->codes || !aligned16(icache->codes) || !icache->scales || !aligned16(icache->scales))
+    return CKV_ERR_INVALID_ARG;
+  if (need_residue && (!icache->residue_k || !aligned16(icache->residue_k) || !icache->residue_logit ||
+                       !aligned16(icache->residue_logit)))
+    return CKV_ERR_INVALID_ARG;
+  ip->heads = H;
+  ip->dim = d;
+  ip->codes = static_cast<uint8_t*>(icache->codes);
+  ip->scales = icache->scales;
+  ip->res_k = icache->residue_k;
+  ip->res_logit = icache->residue_logit;
+  return CKV_OK;
+}
+
+// Workspace of the multi-head indexer: the query images, then the indexer's selection state.
+size_t mh_ws_bytes(const LayerParams& p, const IndexParams& ip, int batch, int max_seq_len, IndexerWs* iw,
+                   uint8_t** qimage, void* base) {
+  const size_t img = mh_image_bytes(ip, batch);
+  *iw = indexer_ws_layout(base ? static_cast<char*>(base) + img : nullptr, p, batch, max_seq_len);
+  if (qimage) *qimage = static_cast<uint8_t*>(base);
+  return img + iw->bytes;
+}
+
 }  // namespace
 }  // namespace ckv
 
@@ -382,6 +412,62 @@ int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int3
   e = launch_attention(p, batch, d_seq_len, max_seq_len, d_q, top_k > 0 ? d_idx : nullptr,
                        top_k > 0 ? d_cnt : nullptr, top_k > 0 ? top_k : 0, d_out, aw, d_status, s,
                        front || top_k > 0);
+  return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+}
+
+int kv_index_append(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, const ckv_index_cfg* icfg,
+                    const ckv_index_cache* icache, int32_t batch, const int32_t* d_prev_len,
+                    const int32_t* d_cu_new, int32_t max_new, int32_t max_seq_len, const float* d_k_new,
+                    const float* d_logit_new, uint32_t* d_status, void* stream) {
+  LayerParams p{};
+  int st = make_params(cfg, cache, batch, max_seq_len, false, &p);
+  if (st != CKV_OK) return st;
+  IndexParams ip{};
+  st = make_index_params(icfg, icache, true, &ip);
+  if (st != CKV_OK) return st;
+  if (!d_prev_len || !d_k_new || !d_logit_new || !d_status || !aligned16(d_k_new)) return CKV_ERR_INVALID_ARG;
+  if (d_cu_new ? max_new < 1 : max_new != 1) return CKV_ERR_INVALID_ARG;
+  cudaError_t e = launch_index_append(p, ip, batch, d_prev_len, d_cu_new, max_new, max_seq_len, d_k_new,
+                                      d_logit_new, d_status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+}
+
+size_t ckv_mh_indexer_workspace_bytes(const ckv_layer_cfg* cfg, const ckv_index_cfg* icfg, int32_t batch,
+                                      int32_t max_seq_len, int32_t top_k) {
+  if (check_cfg(cfg) != CKV_OK || !icfg || batch < 1 || max_seq_len < 1 || top_k < 1) return 0;
+  const int H = icfg->index_heads, d = icfg->index_dim;
+  if (H < 16 || H > 128 || H % 16 != 0 || (d != 128 && d != 256)) return 0;
+  LayerParams p{};
+  p.D = cfg->head_dim;
+  p.r = cfg->ratio;
+  IndexParams ip{};
+  ip.heads = H;
+  ip.dim = d;
+  IndexerWs iw{};
+  return mh_ws_bytes(p, ip, batch, max_seq_len, &iw, nullptr, nullptr);
+}
+
+int sparse_mh_indexer_topk(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, const ckv_index_cfg* icfg,
+                           const ckv_index_cache* icache, int32_t batch, const int32_t* d_seq_len,
+                           int32_t max_seq_len, const float* d_q_index, const float* d_weights, int32_t top_k,
+                           int32_t* d_idx, int32_t* d_cnt, float* d_scores, void* d_ws, size_t ws_bytes,
+                           uint32_t* d_status, void* stream) {
+  LayerParams p{};
+  int st = make_params(cfg, cache, batch, max_seq_len, false, &p);
+  if (st != CKV_OK) return st;
+  IndexParams ip{};
+  st = make_index_params(icfg, icache, false, &ip);
+  if (st != CKV_OK) return st;
+  if (batch > 2048 || p.r > 4) return CKV_ERR_UNSUPPORTED;  // 64-entry runs within one pool block
+  if (!d_seq_len || !d_q_index || !d_weights || !d_idx || !d_cnt || !d_status || top_k < 1 ||
+      !aligned16(d_q_index) || !aligned16(d_idx) || !aligned16(d_cnt) || (d_scores && !aligned16(d_scores)))
+    return CKV_ERR_INVALID_ARG;
+  if (!d_ws || !aligned16(d_ws)) return CKV_ERR_WORKSPACE;
+  IndexerWs iw{};
+  uint8_t* qimage = nullptr;
+  if (ws_bytes < mh_ws_bytes(p, ip, batch, max_seq_len, &iw, &qimage, d_ws)) return CKV_ERR_WORKSPACE;
+  cudaError_t e = launch_mh_indexer(p, ip, batch, d_seq_len, max_seq_len, d_q_index, d_weights, top_k, d_idx,
+                                    d_cnt, d_scores, iw, qimage, d_status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
 }
 

@@ -80,6 +80,32 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
                            cudaStream_t stream, QueryPrepOut prep = {nullptr, nullptr},
                            bool skip_qbar = false);
 
+// Top-k of the scores a score pass wrote, with the candidate counts, the reset selection state
+// and the first-digit histogram in ws (the kernels after the score pass).
+cudaError_t launch_topk(const LayerParams& p, int batch, int max_seq_len, int top_k, const float* scores,
+                        int64_t stride, const IndexerWs& ws, int32_t* idx, int32_t* cnt, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------- multi-head indexer
+// The index plane of a layer: FP8 index entries in the rows of the compressed pool, and the
+// index-key compressor's own residue ring.
+struct IndexParams {
+  int heads;           // H_I: a multiple of 16, 16 .. 128
+  int dim;             // d_I: 128 or 256
+  uint8_t* codes;      // [pool rows][d_I] e4m3
+  float* scales;       // [pool rows] fp32
+  float* res_k;        // [B][r][d_I] fp32
+  float* res_logit;    // [B][r] fp32
+};
+// bytes of the fp16 query images of a batch (the head of the multi-head indexer's workspace)
+size_t mh_image_bytes(const IndexParams& ip, int batch);
+cudaError_t launch_index_append(const LayerParams& p, const IndexParams& ip, int batch, const int32_t* prev_len,
+                                const int32_t* cu_new, int max_new, int max_seq_len, const float* k_new,
+                                const float* logit_new, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_mh_indexer(const LayerParams& p, const IndexParams& ip, int batch, const int32_t* seq_len,
+                              int max_seq_len, const float* q_index, const float* weights, int top_k,
+                              int32_t* idx, int32_t* cnt, float* scores, const IndexerWs& ws,
+                              uint8_t* qimage, uint32_t* status, cudaStream_t stream);
+
 // ---------------------------------------------------------------------------- attention
 struct AttnWs {
   float* part_o;     // [B][S][H][D]   un-normalised partial outputs (CUDA-core path)

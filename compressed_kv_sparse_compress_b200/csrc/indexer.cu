@@ -786,13 +786,17 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
     default: e = cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
+  return launch_topk(p, batch, max_seq_len, top_k, sc, stride, ws, idx, cnt, stream);
+}
+
+cudaError_t launch_topk(const LayerParams& p, int batch, int max_seq_len, int top_k, const float* sc,
+                        int64_t stride, const IndexerWs& ws, int32_t* idx, int32_t* cnt, cudaStream_t stream) {
   const int64_t nmax = static_cast<int64_t>(max_seq_len) / p.r;
   if (nmax <= kSmallMax)   // every request's candidates fit one CTA's registers
-    return launch_kernel(topk_small_kernel, dim3(batch), dim3(kSmallThreads), 0, stream,
-                         static_cast<const float*>(sc), stride, static_cast<int>(nmax), top_k, ws, idx, cnt);
+    return launch_kernel(topk_small_kernel, dim3(batch), dim3(kSmallThreads), 0, stream, sc, stride,
+                         static_cast<int>(nmax), top_k, ws, idx, cnt);
   dim3 mgrid(static_cast<unsigned>(nmax > 0 ? (nmax + kMarkChunk - 1) / kMarkChunk : 1), batch);
-  e = launch_kernel(topk_mark_kernel, mgrid, dim3(kThreads), 0, stream, static_cast<const float*>(sc),
-                    stride, top_k, ws);
+  cudaError_t e = launch_kernel(topk_mark_kernel, mgrid, dim3(kThreads), 0, stream, sc, stride, top_k, ws);
   if (e != cudaSuccess) return e;
   return launch_kernel(topk_finish_kernel, dim3(batch), dim3(kFinishThreads), 0, stream, top_k, ws, stride,
                        idx, cnt);

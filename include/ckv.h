@@ -245,10 +245,6 @@ int sparse_indexer_topk_noalloc(const ckv_layer_cfg* cfg, const ckv_layer_cache*
                                 float* d_scores, uint32_t* d_status, void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
-/* Diagnostics. */
-
-/* Static text of a ckv_status. */
-/* ---------------------------------------------------------------------------------------- */
 /* Fused decode step of one layer: steps 1-3 in one call (the three descriptions above apply).
  * [HR] section A lists the path's parts (compression, top-k over compressed tokens, window,
  * shared K=V attention); [CZ] section C credits the speed-up to fused kernels. One token per
@@ -276,6 +272,72 @@ int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int3
                     int32_t* d_cnt, float* d_out, void* d_ws, size_t ws_bytes, uint32_t* d_status,
                     void* stream);
 
+/* ---------------------------------------------------------------------------------------- */
+/* Multi-head indexer ([CZ] section C: "Sparse MQA logits" scores only the candidate positions).
+ * The pages name the indexer and give no formula; this is its multi-head reading, next to the
+ * head-averaged one of sparse_indexer_topk. The indexer has H_I heads of width d_I and its own
+ * compressed index key per entry:
+ *   - per token the caller supplies an index key (d_I fp32, position encoding already applied;
+ *     the projections that make index keys and queries are outside this library);
+ *   - the keys of a group of r tokens are folded with the softmax weights of the same compressor
+ *     logits as the K=V tokens ([HR] section A: compression by a weighted sum), entry = sum_t w_t
+ *     key_t in fp32, and stored as FP8 e4m3 with one fp32 scale per entry (s = amax / 448, 1 for a
+ *     zero entry; codes = e4m3 RNE-satfinite of x / s: the window's FP8 rule);
+ *   - at decode time each head's index query q_h (d_I fp32) is stored by the same FP8 rule
+ *     (codes q~_h, scale t_h = amax_h / 448) and, with one fp32 weight w_h per head, candidate j
+ *     (an entry < floor(L/r), codes c_j, scale s_j) scores
+ *         score_j = s_j * sum_h (w_h t_h) * max(0, q~_h . c_j)      (e4m3 products, fp32 sums)
+ *     i.e. sum_h w_h max(0, q^_h . k_j) for the decoded query and entry; the top-k rule and
+ *     outputs are those of sparse_indexer_topk.
+ * The index plane lives in the rows of the layer's compressed pool: entry i of request b is row
+ * comp_table[b * table_stride + (i r) / 256] * (256 / r) + i % (256 / r) of `codes` / `scales`. */
+typedef struct {
+  int32_t index_heads; /* H_I: a multiple of 16, 16..128                                   */
+  int32_t index_dim;   /* d_I: 128 or 256                                                  */
+} ckv_index_cfg;
+
+typedef struct {
+  void* codes;          /* d: [comp_blocks][256/r][d_I] e4m3 index entries                 */
+  float* scales;        /* d: [comp_blocks][256/r] fp32 entry scales                       */
+  float* residue_k;     /* d: [batch][r][d_I] fp32 index keys of the unfinished group,
+                           slot = position % r (kv_index_append only)                      */
+  float* residue_logit; /* d: [batch][r] fp32 their logits; a ring of its own, not the
+                           layer's residue_logit (kv_index_append only)                    */
+} ckv_index_cache;
+
+/* Appends n_b index keys to request b at positions prev_len[b] .. prev_len[b]+n_b-1 (the same
+ * tokens, in the same calls, as kv_compress_append): a key whose position + 1 is a multiple of r
+ * completes its group, which is folded and stored as above; the keys of an unfinished group go
+ * to the residue ring. Arguments as for kv_compress_append, with cfg / cache the layer's (ratio,
+ * compressed table and pool size) and d_k_new [sum n_b][d_I] fp32. Nothing outside the index
+ * plane and its ring is written. */
+int kv_index_append(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, const ckv_index_cfg* icfg,
+                    const ckv_index_cache* icache, int32_t batch, const int32_t* d_prev_len,
+                    const int32_t* d_cu_new, int32_t max_new, int32_t max_seq_len, const float* d_k_new,
+                    const float* d_logit_new, uint32_t* d_status, void* stream);
+
+/* Workspace bytes of sparse_mh_indexer_topk (0 on a bad config). */
+size_t ckv_mh_indexer_workspace_bytes(const ckv_layer_cfg* cfg, const ckv_index_cfg* icfg, int32_t batch,
+                                      int32_t max_seq_len, int32_t top_k);
+
+/* Scores every candidate of each request with the multi-head rule and selects the top_k, with the
+ * outputs, padding, tie rule, optional d_scores and device errors of sparse_indexer_topk.
+ *   d_q_index  [batch][H_I][d_I] fp32.   d_weights [batch][H_I] fp32.
+ *   batch      1 .. 2048, ratio r 1, 2 or 4 (256/r >= 64 entries per pool block); otherwise
+ *              CKV_ERR_UNSUPPORTED.
+ *   d_ws       workspace of ws_bytes >= ckv_mh_indexer_workspace_bytes(...).
+ * A wait for the tensor cores that gives up sets CKV_DEV_TIMEOUT (the scores of the tiles not
+ * reached are not written). */
+int sparse_mh_indexer_topk(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, const ckv_index_cfg* icfg,
+                           const ckv_index_cache* icache, int32_t batch, const int32_t* d_seq_len,
+                           int32_t max_seq_len, const float* d_q_index, const float* d_weights, int32_t top_k,
+                           int32_t* d_idx, int32_t* d_cnt, float* d_scores, void* d_ws, size_t ws_bytes,
+                           uint32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* Diagnostics. */
+
+/* Static text of a ckv_status. */
 const char* ckv_status_str(int status);
 /* Number of kernel launches enqueued by this process since load (all entry points). */
 uint64_t ckv_launch_count(void);

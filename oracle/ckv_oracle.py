@@ -543,9 +543,10 @@ def decode_layer(cfg: LayerCfg, cache: LayerCache, b: int, q_raw: np.ndarray, se
 # the index keys of a group are folded with the same softmax weights of the same logits as the
 # K=V tokens ([HR] §A) and stored as FP8 with one fp32 scale per entry (the window's FP8 rule).
 # The decode step supplies one index query per head and one weight per head; the score of
-# candidate j is s_j = sum_h w_h * max(0, q^_h . k_j), where q^ is the index query rounded to
-# fp16 (the precision the scoring takes it in) and k_j the decoded entry. No softmax scale (the
-# weights carry it); top-k as for the head-averaged score.
+# candidate j is s_j = sum_h w_h * max(0, q^_h . k_j), where q^_h is head h's index query stored
+# by the same FP8 rule (one fp32 scale per head: the indexer runs in FP8 end to end, like the
+# pages' FP8/FP4 caches) and k_j the decoded entry. No softmax scale (the weights carry it); top-k
+# as for the head-averaged score.
 # ------------------------------------------------------------------------------------------------
 
 @dataclass(frozen=True)
@@ -605,9 +606,15 @@ def decode_index_entries(cfg: LayerCfg, icache: IndexCache, comp_table: np.ndarr
         icache.scales.reshape(-1)[rows].astype(np.float64)[:, None]
 
 
-def index_query_f16(q_index: np.ndarray) -> np.ndarray:
-    """The index query as scored: each fp32 element rounded to the nearest fp16 (ties to even)."""
-    return np.asarray(q_index, dtype=np.float32).astype(np.float16).astype(np.float64)
+def index_query_fp8(q_index: np.ndarray) -> np.ndarray:
+    """The index query as scored: each head stored by quantize_fp8_token (scale amax/448, e4m3
+    codes), decoded to fp64. q_index: [H_I, d_I]."""
+    q = np.asarray(q_index, dtype=np.float32)
+    out = np.empty(q.shape, dtype=np.float64)
+    for h in range(q.shape[0]):
+        codes, s = quantize_fp8_token(q[h])
+        out[h] = dequant_fp8_token(codes, s)
+    return out
 
 
 def mh_indexer_scores(cfg: LayerCfg, icache: IndexCache, comp_table: np.ndarray, b: int,
@@ -617,7 +624,7 @@ def mh_indexer_scores(cfg: LayerCfg, icache: IndexCache, comp_table: np.ndarray,
 
     q_index: [H_I, d_I] fp32; weights: [H_I] fp32."""
     n_c = num_compressed(seq_len, cfg.ratio)
-    qh = index_query_f16(q_index)
+    qh = index_query_fp8(q_index)
     w = np.asarray(weights, dtype=np.float32).astype(np.float64)
     out = np.empty(n_c, dtype=np.float64)
     for j0 in range(0, n_c, chunk):

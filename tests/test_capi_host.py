@@ -146,3 +146,50 @@ def test_fused_step_workspace_and_argument_checks():
                              None, None, None, None, 0, None, None)
     assert st == ckv.CKV_ERR_INVALID_ARG
     assert ckv.launch_count() == 0
+
+
+def test_mh_indexer_workspace_and_argument_checks():
+    cfg = ckv.LayerConfig(64, 512, 64, 4, 128, "bf16", "fp8")
+    icfg = ckv.IndexConfig(64, 128)
+    ws = ckv.mh_indexer_workspace_bytes(cfg, icfg, 8, 32768, 512)
+    # the FP8 query images (8 x 64 x 128) and scaled head weights (8 x 64 fp32) ahead of the
+    # head-averaged indexer's selection state
+    assert ws == 8 * 64 * 128 + 8 * 64 * 4 + ckv.indexer_workspace_bytes(cfg, 8, 32768, 512)
+    for heads, dim in [(8, 128), (72, 128), (144, 128), (64, 64), (64, 96), (64, 512), (0, 128)]:
+        assert ckv.mh_indexer_workspace_bytes(cfg, ckv.IndexConfig(heads, dim), 8, 32768, 512) == 0
+    assert ckv.mh_indexer_workspace_bytes(cfg, icfg, 8, 32768, 0) == 0
+    lib = ckv.load_library()
+    null_cache = ckv.LayerCacheC()
+    null_icache = ckv.IndexCacheC()
+    st = lib.sparse_mh_indexer_topk(ctypes.byref(cfg.c()), ctypes.byref(null_cache), ctypes.byref(icfg.c()),
+                                    ctypes.byref(null_icache), 1, None, 1024, None, None, 4, None, None, None,
+                                    None, 0, None, None)
+    assert st == ckv.CKV_ERR_INVALID_ARG
+    st = lib.kv_index_append(ctypes.byref(cfg.c()), ctypes.byref(null_cache), ctypes.byref(icfg.c()),
+                             ctypes.byref(null_icache), 1, None, None, 1, 1024, None, None, None, None)
+    assert st == ckv.CKV_ERR_INVALID_ARG
+    # a layer cache that passes the host checks (16-byte aligned host buffers; nothing launches
+    # because the index config is refused first)
+    buf = np.zeros(64, dtype=np.uint8)
+    base = (buf.ctypes.data + 15) // 16 * 16
+    cache = ckv.LayerCacheC(base, None, base, base, base, base, base, base, 8, 1, 1)
+    icache = ckv.IndexCacheC(base, base, base, base)
+    for heads, dim, want in [(72, 128, ckv.CKV_ERR_UNSUPPORTED), (64, 100, ckv.CKV_ERR_UNSUPPORTED)]:
+        st = lib.sparse_mh_indexer_topk(ctypes.byref(cfg.c()), ctypes.byref(cache),
+                                        ctypes.byref(ckv.IndexConfig(heads, dim).c()), ctypes.byref(icache), 1,
+                                        base, 1024, base, base, 4, base, base, None, base, 1 << 30, base, None)
+        assert st == want
+    st = lib.kv_index_append(ctypes.byref(cfg.c()), ctypes.byref(cache), ctypes.byref(icfg.c()),
+                             ctypes.byref(ckv.IndexCacheC(base, base, None, None)), 1, base, None, 1, 1024, base,
+                             base, base, None)
+    assert st == ckv.CKV_ERR_INVALID_ARG  # the append needs the index rings
+    st = lib.sparse_mh_indexer_topk(ctypes.byref(cfg.c()), ctypes.byref(cache), ctypes.byref(icfg.c()),
+                                    ctypes.byref(icache), 4096, base, 1024, base, base, 4, base, base, None,
+                                    base, 1 << 30, base, None)
+    assert st == ckv.CKV_ERR_UNSUPPORTED  # batch above 2048
+    hca = ckv.LayerConfig(64, 512, 64, 128, 128, "bf16", "fp8")
+    st = lib.sparse_mh_indexer_topk(ctypes.byref(hca.c()), ctypes.byref(cache), ctypes.byref(icfg.c()),
+                                    ctypes.byref(icache), 1, base, 1024, base, base, 4, base, base, None,
+                                    base, 1 << 30, base, None)
+    assert st == ckv.CKV_ERR_UNSUPPORTED  # 2 entries per pool block: runs of 64 do not fit
+    assert ckv.launch_count() == 0

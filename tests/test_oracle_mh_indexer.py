@@ -1,9 +1,9 @@
 """Pins of the oracle's multi-head indexer: special cases whose scores are known in closed form.
 
-The multi-head score is s_j = sum_h w_h * max(0, q^_h . k_j) with the index query rounded to fp16
-and k_j an FP8 entry times its scale; the index keys of a group are folded with the softmax of
+The multi-head score is s_j = sum_h w_h * max(0, q^_h . k_j) with each head's index query stored
+as FP8 (scale amax/448) and k_j an FP8 entry times its scale; the index keys of a group are folded with the softmax of
 the group's logits. Each case below fails for one plausible slip: a dropped or misplaced ReLU,
-weights indexed by the wrong axis, a query not rounded (or rounded the wrong way), the entry
+weights indexed by the wrong axis, a query not quantised (or with the wrong scale), the entry
 scale left out, the wrong group or weights in the fold, a residue lost between calls.
 """
 
@@ -45,13 +45,13 @@ def test_one_hot_heads_pick_their_own_weight():
         x = np.zeros(d_i)
         x[j % 16] = 2.0
         _store(ic, table, cfg, 0, j, x, 0.5)
-    c = np.array([1 + h for h in range(16)], dtype=np.float32)         # exact in fp16
+    c = np.array([1 + h for h in range(16)], dtype=np.float32)         # one value per head: exact
     w = np.array([0.25 * (h + 3) for h in range(16)], dtype=np.float32)
     q = np.zeros((16, d_i), dtype=np.float32)
     q[np.arange(16), np.arange(16)] = c
     s = O.mh_indexer_scores(cfg, ic, table, 0, q, w, 4 * n)
     ref = np.array([w[j % 16] * c[j % 16] * 2.0 * 0.5 for j in range(n)])
-    assert np.array_equal(s, ref)
+    assert np.allclose(s, ref, rtol=1e-6, atol=0)   # c_h is 448 times its fp32 scale
 
 
 def test_relu_drops_negative_dots_before_the_weights():
@@ -66,7 +66,8 @@ def test_relu_drops_negative_dots_before_the_weights():
         x = O.e4m3_decode(O.e4m3_encode_satfinite(rng.normal(size=d_i).astype(np.float32) * 4))
         xs.append(x)
         _store(ic, table, cfg, 0, j, x, 1.0)
-    q1 = np.asarray(rng.integers(-8, 9, size=d_i), dtype=np.float32) / 8   # exact in fp16
+    q1 = np.asarray(rng.integers(-8, 9, size=d_i), dtype=np.float32) * 32   # e4m3 values: scale 1 exact
+    q1[0] = 448.0
     q = np.stack([q1, -q1])
     s = O.mh_indexer_scores(cfg, ic, table, 0, q, np.array([1.0, 1.0], np.float32), 32)
     dots = [float(np.dot(q1.astype(np.float64), x)) for x in xs]
@@ -76,19 +77,22 @@ def test_relu_drops_negative_dots_before_the_weights():
     assert np.allclose(s_neg, [-2.0 * max(d, 0.0) for d in dots], rtol=1e-15, atol=0)
 
 
-def test_query_is_rounded_to_fp16_nearest_even():
-    # fp16 has a step of 2^-10 at 1: 1 + 2^-12 rounds down to 1, 1 + 3 * 2^-12 up to 1 + 2^-10,
-    # and 1 + 2^-11 (a tie) to the even neighbour 1
+def test_query_is_stored_as_fp8_per_head():
+    # head 0's query (1, 0.3, 0, ...) has scale 1/448: 0.3 * 448 = 134.4 lies between the e4m3
+    # values 128 and 144 and rounds to 128, so the key e_1 scores 128/448, not 0.3; head 1's query
+    # 0.3 e_1 alone has scale 0.3/448 and is exact. The scale is per head: a shared one would
+    # round head 1 as well
     cfg, d_i = _cfg(), 64
     ic, table = _pool(4, d_i)
     x = np.zeros(d_i)
-    x[0] = 1.0
+    x[1] = 1.0
     _store(ic, table, cfg, 0, 0, x, 1.0)
-    for qv, expect in [(1 + 2.0 ** -12, 1.0), (1 + 3 * 2.0 ** -12, 1 + 2.0 ** -10), (1 + 2.0 ** -11, 1.0)]:
-        q = np.zeros((1, d_i), dtype=np.float32)
-        q[0, 0] = qv
-        s = O.mh_indexer_scores(cfg, ic, table, 0, q, np.array([1.0], np.float32), 4)
-        assert s[0] == expect
+    q = np.zeros((2, d_i), dtype=np.float32)
+    q[0, 0], q[0, 1], q[1, 1] = 1.0, 0.3, 0.3
+    s0 = O.mh_indexer_scores(cfg, ic, table, 0, q[:1], np.array([1.0], np.float32), 4)
+    assert s0[0] == pytest.approx(128.0 / 448.0, rel=1e-6)
+    s1 = O.mh_indexer_scores(cfg, ic, table, 0, q, np.array([0.0, 1.0], np.float32), 4)
+    assert s1[0] == pytest.approx(float(np.float32(0.3)), rel=1e-6)
 
 
 def test_entry_scale_multiplies_the_score():
@@ -99,8 +103,8 @@ def test_entry_scale_multiplies_the_score():
     _store(ic, table, cfg, 0, 1, x, 3.0)
     q = np.ones((2, d_i), dtype=np.float32)
     s = O.mh_indexer_scores(cfg, ic, table, 0, q, np.array([1.0, 0.5], np.float32), 8)
-    assert s[0] == pytest.approx(1.5 * 64 * 0.125, rel=1e-15)
-    assert s[1] == pytest.approx(1.5 * 64 * 3.0, rel=1e-15)
+    assert s[0] == pytest.approx(1.5 * 64 * 0.125, rel=1e-6)
+    assert s[1] == pytest.approx(1.5 * 64 * 3.0, rel=1e-6)
 
 
 def test_all_positive_dots_collapse_to_one_weighted_query():
@@ -116,7 +120,8 @@ def test_all_positive_dots_collapse_to_one_weighted_query():
     q = rng.uniform(0.1, 1.0, size=(8, d_i)).astype(np.float32)
     w = rng.uniform(-1.0, 1.0, size=8).astype(np.float32)
     s = O.mh_indexer_scores(cfg, ic, table, 0, q, w, 256)
-    qbar = (w.astype(np.float64)[:, None] * q.astype(np.float16).astype(np.float64)).sum(axis=0)
+    qhat = np.stack([O.dequant_fp8_token(*O.quantize_fp8_token(qh)) for qh in q])
+    qbar = (w.astype(np.float64)[:, None] * qhat).sum(axis=0)
     ref = np.array([0.25 * float(qbar @ x) for x in xs])
     assert np.allclose(s, ref, rtol=1e-12, atol=1e-12)
 
