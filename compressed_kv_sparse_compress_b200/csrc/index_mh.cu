@@ -179,10 +179,12 @@ __global__ void __launch_bounds__(kIdxAppendThreads) index_append_kernel(IndexAp
 
 constexpr int kMhPrepThreads = 256;
 
-// One CTA per request: candidate count, selection state reset, and the index query of each head
-// stored by the FP8 rule (s_h = amax_h / 448, 1 for a zero head; codes e4m3 of q / s_h) as the
-// K-major operand image: chunk c (dims 128c .. 128c+127) holds H_I rows of 128 bytes, 16-byte
-// granule g of row h stored at slot g ^ (h % 8). The head weights scaled by s_h go to wq.
+// One CTA per (8 heads, request), one warp per head, so that every head's loads are in flight at
+// once: the index query of each head stored by the FP8 rule (s_h = amax_h / 448, 1 for a zero
+// head; codes e4m3 of q / s_h) as the K-major operand image (chunk c = dims 128c .. 128c+127 holds
+// H_I rows of 128 bytes, 16-byte granule g of row h stored at slot g ^ (h % 8)) and the head
+// weights scaled by s_h (wq). The CTAs of head group 0 also set the candidate count and reset the
+// selection state.
 __global__ void __launch_bounds__(kMhPrepThreads) mh_prep_kernel(LayerParams p, IndexParams ip,
                                                                  const int32_t* seq_len, int max_seq_len,
                                                                  const float* q_index, const float* weights,
@@ -190,19 +192,22 @@ __global__ void __launch_bounds__(kMhPrepThreads) mh_prep_kernel(LayerParams p, 
                                                                  uint32_t* status) {
   griddep_wait();
   griddep_launch();
-  const int b = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int L = seq_len[b];
-  const bool ok = L >= 1 && L <= max_seq_len;
-  if (tid == 0) {
-    if (!ok) atomicOr(status, CKV_DEV_BAD_LENGTH);
-    ws.n_c[b] = ok ? L / p.r : 0;
-    ws.cand_cnt[b] = 0;
+  const int b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (blockIdx.x == 0) {
+    const int L = seq_len[b];
+    const bool ok = L >= 1 && L <= max_seq_len;
+    if (tid == 0) {
+      if (!ok) atomicOr(status, CKV_DEV_BAD_LENGTH);
+      ws.n_c[b] = ok ? L / p.r : 0;
+      ws.cand_cnt[b] = 0;
+    }
+    for (int i = tid; i < kHistBins; i += kMhPrepThreads) ws.hist[static_cast<int64_t>(b) * kHistBins + i] = 0;
   }
-  for (int i = tid; i < kHistBins; i += kMhPrepThreads) ws.hist[static_cast<int64_t>(b) * kHistBins + i] = 0;
   const int dI = ip.dim;  // 128 or 256: lane l holds dims [e l, e l + e), e = dI / 32
   const int e = dI / 32;
   uint8_t* img = qimage + static_cast<int64_t>(b) * ip.heads * dI;
-  for (int h = warp; h < ip.heads; h += kMhPrepThreads / 32) {
+  const int h = blockIdx.x * (kMhPrepThreads / 32) + warp;
+  if (h < ip.heads) {
     const float* qh = q_index + (static_cast<int64_t>(b) * ip.heads + h) * dI + e * lane;
     float x[8];
     const float4 v0 = __ldg(reinterpret_cast<const float4*>(qh));
@@ -724,8 +729,9 @@ cudaError_t launch_mh_indexer(const LayerParams& p, const IndexParams& ip, int b
   const int64_t stride = score_stride(p.r, max_seq_len);
   float* sc = scores ? scores : ws.scores;
   float* wq = reinterpret_cast<float*>(qimage + align_up(static_cast<size_t>(batch) * ip.heads * ip.dim, 256));
-  cudaError_t e = launch_kernel(mh_prep_kernel, dim3(batch), dim3(kMhPrepThreads), 0, stream, p, ip, seq_len,
-                                max_seq_len, q_index, weights, ws, qimage, wq, status);
+  const int head_groups = (ip.heads + kMhPrepThreads / 32 - 1) / (kMhPrepThreads / 32);
+  cudaError_t e = launch_kernel(mh_prep_kernel, dim3(head_groups, batch), dim3(kMhPrepThreads), 0, stream, p, ip,
+                                seq_len, max_seq_len, q_index, weights, ws, qimage, wq, status);
   if (e != cudaSuccess) return e;
   switch (ip.dim) {
     case 128: e = launch_mh_score<128>(p, ip, batch, max_seq_len, ws, qimage, wq, sc, stride, status, stream); break;
