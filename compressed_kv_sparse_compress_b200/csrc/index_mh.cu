@@ -238,9 +238,10 @@ __global__ void __launch_bounds__(kMhPrepThreads) mh_prep_kernel(LayerParams p, 
 // ---------------------------------------------------------------------------- scoring
 
 // Warp roles of the score kernel (256 threads): warp 0 lane 0 loads (TMA for the index rows, bulk
-// copies for the query images), warp 1 lane 0 issues the MMAs, warps 4..7 (TMEM lane quarters
-// 0..3, one entry per thread) run the epilogue; warps 2, 3 and the other lanes only take part in
-// the set-up and the final barrier.
+// copies for the entry scales and the query images), warp 1 lane 0 issues the MMAs, warps 4..7
+// (TMEM lane quarters 0..3, one entry per thread) run the epilogue; warp 2 allocates and frees the
+// tensor memory; otherwise warps 2, 3 and the other lanes only take part in the set-up and the
+// final barrier.
 constexpr int kScoreThreads = 256;
 constexpr int kTile = 128;      // entries per tile = MMA M
 constexpr int kBoxRows = 64;    // entries per TMA box (one pool block holds 256 / r >= 64 of them)
