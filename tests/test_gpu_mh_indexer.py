@@ -92,6 +92,20 @@ def test_mh_scores_and_selection_match_the_oracle(cuda_lib, case):
     _check_against_oracle(w, gen, ix, idx, cnt, sc, k)
 
 
+def test_mh_many_short_requests_per_cta(cuda_lib):
+    # 2048 requests of 1 or 2 tiles (every 7th with no candidate): each persistent CTA walks
+    # several requests, so both query-image slots and the per-warp weight slots are reused and the
+    # producer waits for the MMAs of the request two switches back
+    lens = tuple((512 + 100 * (i % 3)) if i % 7 else 3 for i in range(2048))
+    w = S.Workload("mh_2048req", lens, 64, 512, 64, 128, (S.LayerSpec(4, 16, "bf16", "fp8"),),
+                   paged=True, from_scratch=False, seed=7100)
+    gen = S.generate(w, "cuda")
+    ix = S.generate_index(w, gen, device="cuda")
+    idx, cnt, sc, st = _select(cuda_lib, w, gen, ix, 64, 128, 16)
+    assert st == 0, f"status {st:#x}"
+    _check_against_oracle(w, gen, ix, idx, cnt, sc, 16)
+
+
 @pytest.mark.parametrize("lens,k", [((4000, 3001), 50), ((100000, 70001), 300)],
                          ids=["one_cta_selection", "bitmap_selection"])
 def test_mh_zero_query_ties_select_the_lowest_indices(cuda_lib, lens, k):
