@@ -200,3 +200,31 @@ def test_index_entries_land_in_the_paged_rows():
         row = int(table[1][(4 * i) // 256]) * 64 + i % 64
         assert O.e4m3_decode(flat[row:row + 1])[0, 0] * sc[row] == pytest.approx(i + 1, rel=1e-6)
     assert not flat[table[0][0] * 64:(table[0][0] + 1) * 64].any()
+
+
+def test_fp8_query_matches_torchs_e4m3_cast():
+    # library pin of the query quantiser: codes from torch's float8_e4m3fn cast of q / s
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(21)
+    q = rng.normal(size=(16, 128)).astype(np.float32) * rng.uniform(0.01, 100, size=(16, 1)).astype(np.float32)
+    q[3] = 0.0
+    got = O.index_query_fp8(q)
+    for h in range(q.shape[0]):
+        amax = np.float32(np.max(np.abs(q[h])))
+        s = np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+        x = torch.from_numpy(q[h] / s).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        assert np.array_equal(got[h], x * np.float64(s))
+
+
+def test_ratio_one_index_append_stores_each_key():
+    # r = 1: every key is its own group (weight 1), so each entry is the key's FP8 storage
+    cfg, d_i = _cfg(1), 128
+    ic, table = _pool(300, d_i, ratio=1)
+    rng = np.random.default_rng(23)
+    keys = rng.normal(size=(300, d_i)).astype(np.float32)
+    O.index_append_tokens(cfg, ic, table, 0, 0, keys, rng.normal(size=300).astype(np.float32))
+    got = O.decode_index_entries(cfg, ic, table, 0, np.arange(300))
+    for t in range(300):
+        codes, s = O.quantize_fp8_token(keys[t])
+        assert np.array_equal(got[t], O.dequant_fp8_token(codes, s))
+    assert ic.residue[0] == []
