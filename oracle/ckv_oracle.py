@@ -92,7 +92,8 @@ class LayerCfg:
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     """bf16 is the upper 16 bits of a binary32: decode is a 16-bit left shift."""
     u = np.asarray(bits).astype(np.uint16).astype(np.uint32) << np.uint32(16)
-    return u.view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # NaN bit patterns stay NaN; numpy only warns about them
+        return u.view(np.float32).astype(np.float64)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
