@@ -164,3 +164,45 @@ def test_nvfp4_entry_is_45_percent_smaller_than_fp8():
     nvfp4 = d // 2 + d // 16
     fp8 = d + 4
     assert abs((1 - nvfp4 / fp8) - 0.45) < 0.01
+
+
+def _e4m3_code_of_power_of_two(k: int) -> int:
+    """e4m3 code of 2^k from the format's fields (bias 7): normal for k >= -6 (exponent field
+    k + 7, mantissa 0), subnormal below (mantissa 2^(k+9), exponent field 0)."""
+    return (k + 7) << 3 if k >= -6 else 1 << (k + 9)
+
+
+@pytest.mark.parametrize("k", [-9, -7, -6, -3, 0, 1, 5, 8])
+def test_nvfp4_scale_is_the_block_max_over_six(k):
+    """A block whose largest magnitude is 6 * 2^k has the exact scale 2^k: its scale code is the
+    e4m3 code of 2^k and every element is an e2m1 value times 2^k, so each code is that value's
+    own code (6 -> 7, the top finite magnitude). A divisor other than 6 (amax/4 gives the scale
+    1.5 * 2^k and maps 6 * 2^k to the code of 4; amax/5 rounds the scale to 1.25 * 2^k and maps it
+    to 4.8 -> the code of 4) fails both checks."""
+    mags = np.array([6, 4, 3, 2, 1.5, 1, 0.5, 0, 6, 4, 3, 2, 1.5, 1, 0.5, 0], dtype=np.float64)
+    signs = np.array([1, -1] * 8, dtype=np.float64)
+    x = (mags * signs * 2.0 ** k).astype(np.float32)
+    packed, sc = O.quantize_nvfp4(x)
+    assert int(sc[0]) == _e4m3_code_of_power_of_two(k)
+    mag_code = {6: 7, 4: 6, 3: 5, 2: 4, 1.5: 3, 1: 2, 0.5: 1, 0: 0}
+    want = [mag_code[m] | (8 if s < 0 else 0) for m, s in zip(mags, signs)]
+    got = []
+    for byte in packed:
+        got += [int(byte) & 0xF, int(byte) >> 4]
+    # -0 keeps its sign bit (code 8); compare magnitudes there
+    assert [g & 7 for g in got] == [w & 7 for w in want]
+    assert all(g == w for g, w, m in zip(got, want, mags) if m != 0)
+
+
+@pytest.mark.parametrize("k", [-20, -8, 0, 3, 11])
+def test_fp8_token_scale_is_the_token_max_over_448(k):
+    """A token whose largest magnitude is 448 * 2^k has the exact scale 2^k and its largest
+    element the top finite e4m3 code 0x7E (0xFE negative); elements that are e4m3 values times
+    2^k keep their own codes. A divisor of 240 or 256 maps the largest element to 240 or 256
+    (codes 0x77, 0x78) and changes the scale, so both checks fail for it."""
+    vals = np.array([448, -448, 1.0, 0.5, 3.0, -2.0, 0.0, 0.015625], dtype=np.float64)
+    codes_want = [0x7E, 0xFE, 0x38, 0x30, 0x44, 0xC0, 0x00, 0x08]   # 0.015625 = 2^-6: exponent field 1
+    x = (vals * 2.0 ** k).astype(np.float32)
+    codes, s = O.quantize_fp8_token(x)
+    assert s == np.float32(2.0 ** k)
+    assert [int(c) for c in codes] == codes_want
