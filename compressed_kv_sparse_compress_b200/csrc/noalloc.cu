@@ -16,6 +16,8 @@
 // candidate counters) at the start of every call, and calls whose kernels overlap on the GPU
 // (different streams, or different threads without ordering) race on the array.
 
+#include <cuda.h>
+
 #include <mutex>
 
 #include "ckv_internal.h"
@@ -27,22 +29,57 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of g_noalloc_scratch on the current device. In host code the array's name is a
-// host-side stand-in, not a device address; the address a kernel can use comes from
-// cudaGetSymbolAddress, asked once per device with that device current.
+struct ScratchSlot {
+  unsigned long long ctx_id;  // id of the context the address was looked up in (0: none yet)
+  void* addr;
+};
+
+std::mutex g_scratch_mutex;
+ScratchSlot g_scratch[kMaxDevices] = {};
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* f = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(f);
+}
+
+// Device address of g_noalloc_scratch in the current device's current context. In host code the
+// array's name is a host-side stand-in, not a device address; the address a kernel can use comes
+// from cudaGetSymbolAddress, asked with the device current. The answer is kept per device together
+// with the id of the context it was asked in (ids are never reused within a process), and asked
+// again when that context has been replaced (after cudaDeviceReset the module is loaded anew and
+// the array may live elsewhere). Looking up the current context and its id are host-side driver
+// queries that enqueue nothing.
 int scratch_address(void** out) {
+  static const CtxGetCurrentFn get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_ctx || !get_id) return CKV_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CKV_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
+  ScratchSlot& slot = g_scratch[dev];
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return CKV_ERR_CUDA;
+  void* p = nullptr;
+  if (ctx == nullptr) {  // no context yet: the symbol lookup initialises the device's primary one
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return CKV_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return CKV_ERR_CUDA;
   }
-  *out = g_scratch_addr[dev];
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return CKV_ERR_CUDA;
+  if (slot.ctx_id != id || slot.addr == nullptr) {
+    if (p == nullptr && (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr))
+      return CKV_ERR_CUDA;
+    slot.ctx_id = id;
+    slot.addr = p;
+  }
+  *out = slot.addr;
   return CKV_OK;
 }
 

@@ -235,7 +235,10 @@ int compressed_window_attention(const ckv_layer_cfg* cfg, const ckv_layer_cache*
  * CKV_ERR_WORKSPACE before anything is enqueued. No allocation of any kind is made.
  *
  * The first call on a device looks up the array's device address on that device (a host-side
- * runtime query, no allocation); make that first call before any stream capture. All calls share
+ * runtime query, no allocation); make that first call before any stream capture. Later calls only
+ * check, with host-side driver queries, that the device's context is still the one the address
+ * was found in; the first call after the context was replaced (cudaDeviceReset) looks it up again
+ * and should also come before any stream capture. All calls share
  * the array and it keeps the last call's contents: the kernels reset the parts that must start at
  * zero on every call, and calls whose kernels overlap on the GPU (other streams, or unordered
  * threads) race on it. */
