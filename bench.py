@@ -6,9 +6,15 @@ token through the compressor (position L-1; idempotent across steps), score ever
 entry and select the top-k (sparse layers), attend over the selected entries plus the window.
 Inputs are resident in HBM; L2 is flushed before every timed step, outside the step's events:
 a 256 MiB buffer is written, then another 256 MiB buffer is read, so that the flush's dirty lines
-are written back before the step starts instead of during it. The metric is decode-attention queries*layers per second over all ranks.
+are written back before the step starts instead of during it. The metric is decode-attention
+queries*layers per second over all ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ckv|reference]
+
+The headline workload is the 1M-context CSA layer (batch 4, the largest configuration that fits
+one GPU). At N = 1 the same line also carries `per_config`: every named configuration (4K fp32,
+32K, 128K HCA, 1M, mixed 64 requests) measured the same way, each with the indexer's and the
+attention's roofline and its own end-to-end figure.
 
 For N > 1 launch one rank per GPU with torch.distributed.run; every rank runs its own batch of
 the workload (data-parallel requests, no collective on the data path) and rank 0 prints one JSON
@@ -38,7 +44,8 @@ from synth import workloads as S  # noqa: E402
 
 METRIC = "decode attention queries*layers/s"
 UNIT = "queries*layers/s"
-DEFAULT_WORKLOAD = "csa_b8_ctx32k"
+DEFAULT_WORKLOAD = "csa_b4_ctx1m"
+CONFIGS = ("csa_b1_ctx4k_fp32", "csa_b8_ctx32k", "hca_b32_ctx128k", "csa_b4_ctx1m", "mixed_64req")
 FLUSH_BYTES = 256 << 20
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
@@ -61,8 +68,9 @@ MH_HEADS, MH_DIM = 64, 128  # multi-head indexer: index heads x index dim
 
 def layer_bytes(w: S.Workload, ls: S.LayerSpec, indexer: str = "avg") -> dict:
     """Bytes a step must move for one layer: the indexer reads every candidate once (its K=V
-    entry for the head-averaged score; its FP8 index entry and scale for the multi-head score);
-    attention reads the selected entries, the window tokens, the query and writes the output; the
+    entry for the head-averaged score; its FP8 index entry and scale for the multi-head score)
+    and the block-table entry of each 256-token block; attention reads the selected entries, the
+    window tokens, the query and writes the output; the
     append reads the unfinished group's ring and writes one entry and one window token (the
     multi-head form also appends the index key: its ring, one FP8 entry)."""
     d, h = w.head_dim, w.num_heads
@@ -74,7 +82,7 @@ def layer_bytes(w: S.Workload, ls: S.LayerSpec, indexer: str = "avg") -> dict:
                 idx_b += n_c * (MH_DIM + 4) + 4 * math.ceil(L / 256) + 4 * MH_HEADS * (MH_DIM + 1)
                 app_b += 4 * MH_DIM + 4 + (ls.ratio - 1) * (4 * MH_DIM + 4) + MH_DIM + 4
             else:
-                idx_b += n_c * entry_bytes(ls, d) + 4 * math.ceil(L / 256) + 4 * h * d
+                idx_b += n_c * entry_bytes(ls, d) + 4 * math.ceil(L / 256)
             sel = min(ls.top_k, n_c)
         else:
             sel = n_c
@@ -273,20 +281,45 @@ class Step:
         return max(int(dl.status[0].item()) & 0xffffffff for dl, _ in self.layers)
 
 
-def run_cuda(args, w: S.Workload):
-    import compressed_kv_sparse_compress_b200 as ckv
-    ckv.load_library()
-    ws, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if ws > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=dev)
+def roofline_record(kind: str, bytes_per_launch: float, launch_ms: list, peak: float, peak_src: str,
+                    workload: str, flops_per_launch: float | None = None, note: str = "") -> dict:
+    """Achieved bandwidth of one kernel kind: algorithmic bytes per launch over the average
+    CUDA-event duration of its launches, against the peak."""
+    avg_ms = sum(launch_ms) / len(launch_ms)
+    ach = bytes_per_launch / (avg_ms / 1e3) / 1e9
+    rec = {"bound": "hbm", "kernel": kind, "achieved": ach, "peak": peak, "peak_source": peak_src,
+           "unit": "GB/s", "frac": ach / peak, "frac_of_8TBps": ach / 8000.0,
+           "avg_launch_us": avg_ms * 1e3, "algorithmic_bytes": bytes_per_launch,
+           "launches_timed": len(launch_ms), "timed_in": note,
+           "traffic": traffic_record(kind, workload)}
+    if flops_per_launch is not None:
+        try:
+            with open(PEAKS_FILE) as f:
+                tpk, tsrc = float(json.load(f)["bf16_tflops"]), "measured bf16 burst"
+        except Exception:
+            tpk, tsrc = 1590.0, "fallback"
+        tf = flops_per_launch / (avg_ms / 1e3) / 1e12
+        rec["tensor"] = {"flops_per_launch": flops_per_launch, "achieved_tflops": tf, "peak_tflops": tpk,
+                         "peak_source": tsrc, "frac": tf / tpk}
+    return rec
+
+
+def attention_flops(w: S.Workload, ls: S.LayerSpec) -> float:
+    """Algorithmic tensor work of one layer's attention: 2 H D flops per key for the logits and
+    2 H D per key for the weighted sum."""
+    keys = 0
+    for L in w.seq_lens:
+        n_c = L // ls.ratio
+        keys += (min(ls.top_k, n_c) if ls.top_k is not None else n_c) + min(w.window, L)
+    return 4.0 * w.num_heads * w.head_dim * keys
+
+
+def measure(ckv, args, w: S.Workload, dev, ws: int, rank: int, cpu_leg: bool) -> dict:
+    """Every timed figure of one workload on this rank (max over ranks where it matters)."""
     step = Step(ckv, w, seed_offset=rank, api=args.api, indexer=args.indexer)
     flush_w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_sink = torch.empty(1, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def flush_l2():
@@ -300,31 +333,23 @@ def run_cuda(args, w: S.Workload):
         torch.cuda.synchronize()
 
     sparse = any(ls.top_k is not None for ls in w.layers)
-    dominant = "attention_kernel" if not sparse else ("mh_score_kernel" if args.indexer == "mh" else "score_kernel")
-    prof_which = ckv.CKV_PROF_ATTENTION if dominant == "attention_kernel" else ckv.CKV_PROF_SCORE
-    n_dom = sum(1 for ls in w.layers if (ls.top_k is not None) == (dominant != "attention_kernel"))
+    score_name = "mh_score_kernel" if args.indexer == "mh" else "score_kernel"
+    dominant = score_name if sparse else "attention_kernel"
 
     for _ in range(args.warmup):
         flush_l2()
         step.run()
     barrier()
     if step.status() != 0:
-        raise RuntimeError(f"device status {step.status():#x} after warm-up")
+        raise RuntimeError(f"device status {step.status():#x} after warm-up ({w.name})")
 
-    # ---- timed region: K steps with one event pair per step. Events between kernels end the
-    #      programmatic launch overlap of the kernels they separate, so the dominant kernel is timed
-    #      in a second pass of K steps with an event pair around each of its launches.
+    # ---- timed region: K steps with one event pair per step, the step replayed as one CUDA graph
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(n_dom)] for _ in range(args.steps)]
-    kstep = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps)]
-    for pair in ev + kstep + [x for row in kev for x in row]:  # CUDA events are created on first record
+    for pair in ev:  # CUDA events are created on first record
         for e in pair:
             e.record(stream)
     torch.cuda.synchronize()
-    # the step (every layer's calls) as one CUDA graph, replayed once per timed step
     step_graph, step_launch = None, "eager"
     launches_per_step = None
     if not args.no_graph:
@@ -340,8 +365,6 @@ def run_cuda(args, w: S.Workload):
         except RuntimeError as exc:   # capture refused: stay eager and say so
             step_launch = "eager (graph capture failed: %s)" % str(exc).splitlines()[0][:120]
             torch.cuda.synchronize()
-    clocks = ClockSampler(local)
-    time.sleep(0.3)
     launches0 = ckv.launch_count()
     barrier()
     for i in range(args.steps):
@@ -355,34 +378,58 @@ def run_cuda(args, w: S.Workload):
     barrier()
     launches = (launches_per_step * args.steps if step_graph is not None
                 else ckv.launch_count() - launches0)
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(step_ms), dev)
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
 
-    barrier()
-    for i in range(args.steps):
-        flush_l2()
-        kstep[i][0].record(stream)
-        if n_dom == 1:
-            ckv.profile_events(prof_which, kev[i][0][0], kev[i][0][1])
-            step.run()
-        else:  # one event pair per layer of the dominant kind
+    # ---- kernel passes: events between kernels end the programmatic launch overlap of the
+    #      kernels they separate, so each kernel kind is timed in a pass of K steps of its own, with
+    #      an event pair around every launch of that kind
+    def kernel_pass(which, takes):
+        pairs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for li in range(len(w.layers)) if takes(w.layers[li])] for _ in range(args.steps)]
+        kst = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            flush_l2()
+            kst[i][0].record(stream)
             k = 0
-            for li, (dl, lay) in enumerate(step.layers):
-                is_dom = (dl.top_k is not None) == (dominant != "attention_kernel")
-                if is_dom:
-                    ckv.profile_events(prof_which, kev[i][k][0], kev[i][k][1])
+            for li in range(len(w.layers)):
+                if takes(w.layers[li]):
+                    ckv.profile_events(which, pairs[i][k][0], pairs[i][k][1])
                     k += 1
                 else:
-                    ckv.profile_events(prof_which)
+                    ckv.profile_events(which)
                 step.run_layer(li, step.seq, step.prev, step.inputs(li))
-        kstep[i][1].record(stream)
-    barrier()
-    ckv.profile_events(prof_which)
-    clk = clocks.stop()
-    dom_ms = [a.elapsed_time(b) for row in kev for a, b in row]
-    kstep_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in kstep), dev)
+            kst[i][1].record(stream)
+        barrier()
+        ckv.profile_events(which)
+        # per step: the summed duration of this kind's launches (one per layer of the kind)
+        per_step = [sum(a.elapsed_time(b) for a, b in row) for row in pairs]
+        step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in kst), dev) / args.steps
+        return per_step, step_ms, len(pairs[0])
+
+    peak, peak_src = measured_peak()
+    lb = [layer_bytes(w, ls, args.indexer) for ls in w.layers]
+    rooflines = {}
+    if sparse:
+        per_step, sms, n = kernel_pass(ckv.CKV_PROF_SCORE, lambda ls: ls.top_k is not None)
+        idx_bytes = sum(b["indexer"] for b, ls in zip(lb, w.layers) if ls.top_k is not None)
+        rooflines["indexer"] = roofline_record(
+            score_name, idx_bytes, per_step, peak, peak_src, w.name,
+            note=f"a pass of K steps with an event pair around each launch of the score kernel "
+                 f"({n} per step; bytes and time summed over them; that pass: {sms * 1e3:.1f} us per step)")
+        if args.indexer == "mh":
+            rooflines["indexer"]["tensor"] = tensor_record(w, args.indexer, sum(per_step) / len(per_step))
+    per_step, sms, n = kernel_pass(ckv.CKV_PROF_ATTENTION, lambda ls: True)
+    att_bytes = sum(b["attention"] for b in lb)
+    rooflines["attention"] = roofline_record(
+        "attention_kernel", att_bytes, per_step, peak, peak_src, w.name,
+        flops_per_launch=sum(attention_flops(w, ls) for ls in w.layers),
+        note=f"a pass of K steps with an event pair around the attention kernel and its split merge "
+             f"of every layer ({n} per step; bytes and time summed over them; that pass: "
+             f"{sms * 1e3:.1f} us per step)")
     if step.status() != 0:
-        raise RuntimeError(f"device status {step.status():#x} in the timed region")
+        raise RuntimeError(f"device status {step.status():#x} in the timed region ({w.name})")
 
     # ---- end to end through the public API: pinned host inputs -> device -> result on host
     ins_h = [[x.cpu().pin_memory() for x in step.inputs(i)] for i in range(len(step.layers))]
@@ -408,7 +455,6 @@ def run_cuda(args, w: S.Workload):
         flush_l2()
         e2e_step()
     barrier()
-    # the whole end-to-end step (copies in, every layer's call, copy out) as one CUDA graph
     run_e2e, graph_note = e2e_step, "eager"
     if not args.no_graph:
         try:
@@ -432,21 +478,10 @@ def run_cuda(args, w: S.Workload):
     barrier()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev), dev)
 
-    units = w.batch * len(w.layers) * ws  # queries*layers per step over all ranks
-    value = job_throughput(w.batch * len(w.layers), ws, args.steps, total_ms)
-    peak, peak_src = measured_peak()
-    lb = [layer_bytes(w, ls, args.indexer) for ls in w.layers]
-    if dominant != "attention_kernel":
-        dom_bytes = sum(b["indexer"] for b, ls in zip(lb, w.layers) if ls.top_k is not None) / n_dom
-    else:
-        dom_bytes = sum(b["attention"] for b, ls in zip(lb, w.layers) if ls.top_k is None) / n_dom
-    dom_avg_ms = sum(dom_ms) / len(dom_ms)
-    achieved = dom_bytes / (dom_avg_ms / 1e3) / 1e9
+    units = w.batch * len(w.layers)  # queries*layers per step on this rank
     step_bytes = sum(sum(b.values()) for b in lb)
-    result = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+    rec = {
+        "value": job_throughput(units, ws, args.steps, total_ms), "ms_per_step": total_ms / args.steps,
         "config": {
             "workload": w.name, "batch_per_gpu": w.batch, "seq_lens": summarize_lens(w.seq_lens),
             "heads": w.num_heads, "head_dim": w.head_dim, "rope_dim": w.rope_dim,
@@ -456,12 +491,12 @@ def run_cuda(args, w: S.Workload):
             "paged": w.paged, "parallelism": f"dp{ws} (independent requests per GPU)",
             "l2": "flushed before every step outside the step events: 256 MiB written, then another "
                   "256 MiB read (the written lines are evicted before the step)",
-            "step": "append decode token + indexer/top-k + attention (+ split combine), per layer",
+            "step": "append decode token + indexer/top-k + attention (+ split merge), per layer",
             "api": ("kv_compress_append + kv_index_append + sparse_mh_indexer_topk + "
                     "compressed_window_attention on sparse layers" if args.indexer == "mh"
                     else "ckv_decode_step, one call per layer" if args.api == "fused"
                     else "kv_compress_append + sparse_indexer_topk + compressed_window_attention"),
-            "indexer": (f"multi-head: {MH_HEADS} index heads x {MH_DIM} dims, FP8 index entries, fp16 query"
+            "indexer": (f"multi-head: {MH_HEADS} index heads x {MH_DIM} dims, FP8 index entries and query"
                         if args.indexer == "mh" else "head-averaged MQA logits over the K=V entries"),
             "launch": step_launch,
         },
@@ -469,25 +504,67 @@ def run_cuda(args, w: S.Workload):
                 "step_GBps": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
                 "frac_of_measured": step_bytes / (total_ms / args.steps / 1e3) / 1e9 / peak,
                 "frac_of_8TBps": step_bytes / (total_ms / args.steps / 1e3) / 1e9 / 8000.0},
-        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
-                     "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
-                     "avg_launch_us": dom_avg_ms * 1e3, "algorithmic_bytes": dom_bytes,
-                     "launches_timed": len(dom_ms),
-                     "timed_in": "a second pass of K steps with an event pair around every launch "
-                                 "of the kernel (that pass: %.1f us per step)" % (kstep_ms / args.steps * 1e3),
-                     "traffic": traffic_record(dominant, w.name)},
-        "tensor": tensor_record(w, args.indexer, dom_avg_ms) if dominant == "mh_score_kernel" else None,
-        "e2e": {"value": job_throughput(w.batch * len(w.layers), ws, args.steps, e2e_ms), "unit": UNIT,
+        "roofline": dict(rooflines["indexer" if sparse else "attention"]),
+        "roofline_indexer": rooflines.get("indexer"),
+        "roofline_attention": rooflines["attention"],
+        "e2e": {"value": job_throughput(units, ws, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "launch": graph_note,
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": launches,
-        "clocks": clk,
     }
+    assert rec["roofline"]["kernel"] == dominant
+    if cpu_leg:
+        rec["cpu_baseline"] = cpu_baseline(w, step, args.cpu_seconds)
+    del step, step_graph, ev
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_cuda(args, w: S.Workload):
+    import compressed_kv_sparse_compress_b200 as ckv
+    ckv.load_library()
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    cpu_leg = rank == 0 and ws == 1 and not args.no_cpu_baseline
+    head = measure(ckv, args, w, dev, ws, rank, cpu_leg)
+    per_config = None
+    if ws == 1 and not args.no_per_config:
+        per_config = {}
+        for name in CONFIGS:
+            wc = S.WORKLOADS[name]()
+            if wc.name == w.name:
+                rec = dict(head)
+                rec.pop("cpu_baseline", None)
+            else:
+                rec = measure(ckv, args, wc, dev, ws, rank, False)
+            per_config[name] = {k: rec[k] for k in ("value", "ms_per_step", "roofline_indexer",
+                                                    "roofline_attention", "e2e", "gpu_launches")}
+            per_config[name]["workload"] = wc.name
+            per_config[name]["hbm_step_frac_of_measured"] = rec["hbm"]["frac_of_measured"]
+    clk = clocks.stop()
+    result = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": head["config"], "hbm": head["hbm"], "roofline": head["roofline"],
+        "roofline_indexer": head["roofline_indexer"], "roofline_attention": head["roofline_attention"],
+        "tensor": (head["roofline_indexer"] or {}).get("tensor") if args.indexer == "mh" else None,
+        "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": clk,
+    }
+    if "cpu_baseline" in head:
+        result["cpu_baseline"] = head["cpu_baseline"]
+    if per_config is not None:
+        result["per_config"] = per_config
     if ws > 1:
         torch.distributed.barrier()
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, step, args.cpu_seconds)
-    if ws > 1:
         torch.distributed.destroy_process_group()
     return result if rank == 0 else None
 
@@ -510,6 +587,24 @@ def oracle_threads() -> int:
         return max(n) if n else 1
     except Exception:
         return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    """The host CPU's model name as lscpu prints it (else /proc/cpuinfo's)."""
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def oracle_request(w, gen_host, li, b, O, ix_host=None):
@@ -551,26 +646,38 @@ def index_host(ix):
 
 
 def cpu_baseline(w, step, seconds):
+    """The oracle on the host cores, on a bounded sample of the workload's requests (the same
+    seeded inputs): once limited to one thread, once with every thread numpy's pool has."""
+    from threadpoolctl import threadpool_limits
     from oracle import ckv_oracle as O
     gen_host = host_inputs(step.gen)
     ix_host = [index_host(None if mh is None else mh["ix"]) for mh in step.index]
-    done = 0
-    t0 = time.perf_counter()
-    reqs = []
-    while True:
-        for li in range(len(w.layers)):
-            b = done % w.batch
-            oracle_request(w, gen_host, li, b, O, ix_host[li])
-            reqs.append((li, b))
-        done += 1
-        if time.perf_counter() - t0 >= seconds or done >= 64 * w.batch:
-            break
-    el = time.perf_counter() - t0
-    return {"value": done * len(w.layers) / el, "unit": UNIT, "cores": oracle_threads(),
-            "kind": "oracle",
-            "sample": f"{done} requests x {len(w.layers)} layer(s) of {w.name} (same seeded inputs), "
-                      f"each a full append+select+attend in the fp64 numpy oracle"
-                      f"{' with the multi-head indexer' if step.indexer == 'mh' else ''}; {el:.1f} s"}
+
+    def leg(budget):
+        done = 0
+        t0 = time.perf_counter()
+        while True:
+            for li in range(len(w.layers)):
+                oracle_request(w, gen_host, li, done % w.batch, O, ix_host[li])
+            done += 1
+            if time.perf_counter() - t0 >= budget or done >= 64 * w.batch:
+                break
+        el = time.perf_counter() - t0
+        return done * len(w.layers) / el, done, el
+
+    with threadpool_limits(limits=1):
+        v1, n1, t1 = leg(seconds / 2)
+    threads = oracle_threads()
+    vall, nall, tall = leg(seconds / 2)
+    what = (f"requests x {len(w.layers)} layer(s) of {w.name} (same seeded inputs), each a full "
+            f"append+select+attend in the fp64 numpy oracle"
+            f"{' with the multi-head indexer' if step.indexer == 'mh' else ''}")
+    return {"value": vall, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{nall} {what}; {tall:.1f} s on {threads} threads",
+            "one_thread": {"value": v1, "unit": UNIT, "cores": 1, "sample": f"{n1} {what}; {t1:.1f} s"},
+            "all_threads": {"value": vall, "unit": UNIT, "cores": threads,
+                            "sample": f"{nall} {what}; {tall:.1f} s"},
+            "nproc": os.cpu_count(), "cpu_model": cpu_model()}
 
 
 def run_reference(args, w):
@@ -605,7 +712,8 @@ def run_reference(args, w):
         "config": {"workload": w.name, "sample_requests_per_step": per_step, "indexer": args.indexer,
                    "note": "CPU oracle (fp64 numpy) on a bounded sample of the workload's requests"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                         "sample": f"{per_step} request(s) x {len(w.layers)} layer(s) per step"},
+                         "sample": f"{per_step} request(s) x {len(w.layers)} layer(s) per step",
+                         "nproc": os.cpu_count(), "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -624,8 +732,10 @@ def main():
                          f"({MH_HEADS} heads x {MH_DIM} dims) over its own FP8 index entries")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-graph", action="store_true", help="end-to-end steps launched eagerly")
-    ap.add_argument("--reference-requests", type=int, default=0,
+    ap.add_argument("--no-graph", action="store_true", help="steps launched eagerly, not as CUDA graphs")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="measure only --workload (by default N = 1 also measures every named config)")
+    ap.add_argument("--reference-requests", type=int, default=1,
                     help="requests of the batch the reference arm runs per step (0: all)")
     args = ap.parse_args()
     w = S.WORKLOADS[args.workload]()

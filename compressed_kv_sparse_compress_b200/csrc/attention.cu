@@ -477,7 +477,6 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
       default: return cudaErrorInvalidValue;
     }
   }
-  prof_end(kProfAttention, stream);
   if (e != cudaSuccess) return e;
   dim3 grid(p.H, batch);
   if (ws.half_parts) {   // tensor-core path: H = 64, D = 512
@@ -485,12 +484,15 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
     const int smem = gs * static_cast<int>(kGRow);
     e = allow_smem(reinterpret_cast<const void*>(attn_combine_tc_kernel), smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(attn_combine_tc_kernel, dim3(p.H / kGH, batch), dim3(kGThreads), smem, stream, p,
-                         seq_len, max_seq_len, cnt, idx != nullptr, idx_stride, gs, ws, out, status);
+    e = launch_kernel(attn_combine_tc_kernel, dim3(p.H / kGH, batch), dim3(kGThreads), smem, stream, p,
+                      seq_len, max_seq_len, cnt, idx != nullptr, idx_stride, gs, ws, out, status);
+  } else {
+    const dim3 block(p.D / 2);   // one thread per pair of dims: 32 .. 512
+    e = launch_kernel(attn_combine_kernel, grid, block, 0, stream, p, seq_len, max_seq_len, cnt,
+                      idx != nullptr, idx_stride, ws, out, status);
   }
-  const dim3 block(p.D / 2);   // one thread per pair of dims: 32 .. 512
-  return launch_kernel(attn_combine_kernel, grid, block, 0, stream, p, seq_len, max_seq_len, cnt,
-                       idx != nullptr, idx_stride, ws, out, status);
+  prof_end(kProfAttention, stream);   // the attention step: its kernel and the split combine
+  return e;
 }
 
 }  // namespace ckv

@@ -599,10 +599,11 @@ cudaError_t launch_tc(const LayerParams& p, int batch, const int32_t* seq_len, i
 
 }  // namespace
 
+// fp32 caches stay on the CUDA-core path: their values are neither exact in fp16 nor inside its
+// range, and fp32 arithmetic attends them as stored
 bool attention_tc_supported(const LayerParams& p) {
-  return p.H == kH && p.D == kD &&
-         (p.comp_dtype == CKV_BF16 || p.comp_dtype == CKV_NVFP4 || p.comp_dtype == CKV_F32) &&
-         (p.win_dtype == CKV_FP8_E4M3 || p.win_dtype == CKV_F32);
+  return p.H == kH && p.D == kD && (p.comp_dtype == CKV_BF16 || p.comp_dtype == CKV_NVFP4) &&
+         p.win_dtype == CKV_FP8_E4M3;
 }
 
 int attention_tc_tiles_per_split(int batch, int64_t max_keys) {
@@ -629,10 +630,6 @@ cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* 
     return launch_tc<CT, WT>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);
   CKV_TC(CKV_BF16, CKV_FP8_E4M3)
   CKV_TC(CKV_NVFP4, CKV_FP8_E4M3)
-  CKV_TC(CKV_F32, CKV_FP8_E4M3)
-  CKV_TC(CKV_BF16, CKV_F32)
-  CKV_TC(CKV_NVFP4, CKV_F32)
-  CKV_TC(CKV_F32, CKV_F32)
 #undef CKV_TC
   return cudaErrorInvalidValue;
 }

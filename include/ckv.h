@@ -348,7 +348,8 @@ uint64_t ckv_launch_count(void);
 /* Diagnostic timing. While set, every later call records the CUDA events ev_begin (just before)
  * and ev_end (just after) the launch of one kernel, on the call's stream:
  *   CKV_PROF_SCORE      the scoring kernel of sparse_indexer_topk
- *   CKV_PROF_ATTENTION  the attention kernel of compressed_window_attention (before the combine)
+ *   CKV_PROF_ATTENTION  the attention kernels of compressed_window_attention (the attention
+ *                       kernel and the merge of its splits, which writes the output)
  * ev_begin / ev_end are cudaEvent_t handles created by the caller; NULL, NULL stops recording.
  * Process-wide setting, not thread-safe. Returns CKV_ERR_INVALID_ARG for an unknown `which` or
  * only one NULL handle. */

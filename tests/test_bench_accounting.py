@@ -19,8 +19,10 @@ def test_head_averaged_indexer_reads_every_entry_once():
     ls = w.layers[0]
     b = bench.layer_bytes(w, ls)
     n_c = 32768 // 4
-    # bf16 entries of 512 dims, the block table of each request, the raw query [64][512] fp32
-    assert b["indexer"] == 8 * (n_c * 1024 + 4 * 128 + 4 * 64 * 512)
+    # bf16 entries of 512 dims and the block table of each request (the score kernel reads the
+    # head-averaged query; the raw [64][512] query is read by the query pass before it)
+    assert b["indexer"] == 8 * (n_c * 1024 + 4 * 128)
+    assert b["indexer"] == 67112960
     # attention: 512 selected entries + 128 FP8 window tokens (512 codes + a scale) + q in, o out
     assert b["attention"] == 8 * (512 * 1024 + 128 * (512 + 4) + 2 * 4 * 64 * 512)
 
@@ -52,3 +54,27 @@ def test_multi_head_tensor_record_counts_two_flops_per_head_dim_and_entry():
     assert r["flops_per_launch"] == flops
     assert r["achieved_tflops"] == pytest.approx(flops / 1e-5 / 1e12)
     assert r["frac"] == pytest.approx(r["achieved_tflops"] / r["peak_tflops"])
+
+
+def test_attention_flops_count_both_products_per_key():
+    w = S.csa_b4_ctx1m()
+    # 2048 selected entries + 128 window tokens per request, 2 H D flops each for the logits and
+    # for the weighted sum
+    assert bench.attention_flops(w, w.layers[0]) == 4 * 4.0 * 64 * 512 * (2048 + 128)
+    h = S.hca_b32_ctx128k()
+    assert bench.attention_flops(h, h.layers[0]) == 32 * 4.0 * 64 * 512 * (1024 + 128)
+
+
+def test_roofline_record_divides_bytes_by_the_average_launch():
+    r = bench.roofline_record("attention_kernel", 1e9, [1.0, 3.0], 6425.6, "measured", "none",
+                              flops_per_launch=2e12)
+    assert r["achieved"] == pytest.approx(1e9 / 2e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6425.6)
+    assert r["tensor"]["achieved_tflops"] == pytest.approx(2e12 / 2e-3 / 1e12)
+    assert r["traffic"] is None
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    assert bench.DEFAULT_WORKLOAD == "csa_b4_ctx1m"
+    assert set(bench.CONFIGS) == {"csa_b1_ctx4k_fp32", "csa_b8_ctx32k", "hca_b32_ctx128k", "csa_b4_ctx1m",
+                                  "mixed_64req"}
