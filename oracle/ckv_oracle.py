@@ -459,6 +459,40 @@ def append_tokens(cfg: LayerCfg, cache: LayerCache, b: int, prev_len: int,
 
 
 # ------------------------------------------------------------------------------------------------
+# SWA bounded replay ([CZ] §A "Proč je obnova sliding-window cache drahá": after a prefix-cache hit
+# only the last window is run through the model again, and at its start the dependence on older
+# positions is cut; §B "Polovina vrstev nemusí číst celý prompt" names the switch that enables it).
+# The model's recompute of the window's K=V vectors lies outside this path; the cache side is:
+# reading: the caller supplies the recomputed raw tokens and compressor logits of the last
+# n_w = min(W, L) positions; each is rotated at its own position and written to the window cache;
+# the tokens of the unfinished group [floor(L/r) r, L) that lie in the window become the residue
+# (tokens of that group before L - n_w, possible only when r - 1 > W, keep whatever residue state
+# they had: the cut); compressed entries are not touched (they come from the prefix cache).
+# ------------------------------------------------------------------------------------------------
+
+def window_replay(cfg: LayerCfg, cache: LayerCache, b: int, seq_len: int, kv_win: np.ndarray,
+                  logit_win: np.ndarray) -> None:
+    """Rewrite request b's window and residue from the raw tokens of positions L-n_w .. L-1.
+
+    kv_win: [n_w, D] fp32 raw (un-rotated) tokens, row i at position L - n_w + i; logit_win: [n_w]."""
+    n_w = min(cfg.window, seq_len)
+    kv_win = np.asarray(kv_win, dtype=np.float32).reshape(-1, cfg.head_dim)[:n_w]
+    logit_win = np.asarray(logit_win, dtype=np.float32).reshape(-1)[:n_w]
+    g0 = (seq_len // cfg.ratio) * cfg.ratio  # first position of the unfinished group
+    while len(cache.residue) <= b:
+        cache.residue.append([])
+    kept = [e for e in cache.residue[b] if g0 <= e[0] < seq_len - n_w]
+    res = list(kept)
+    for i in range(n_w):
+        pos = seq_len - n_w + i
+        x = rope_apply(kv_win[i].astype(np.float64), pos, cfg.rope_dim, cfg.base)
+        write_window_token(cfg, cache, b, pos, x.astype(np.float32))
+        if pos >= g0:
+            res.append((pos, kv_win[i].copy(), np.float32(logit_win[i])))
+    cache.residue[b] = sorted(res, key=lambda e: e[0])
+
+
+# ------------------------------------------------------------------------------------------------
 # Step 2: sparse MQA indexer and top-k ([HR] §A: sparse attention over the top-k compressed
 # tokens; [CZ] §C: "Sparse MQA logits" scores the candidate positions).
 # reading: the score of candidate j is the head-average of the MQA attention logits of the
