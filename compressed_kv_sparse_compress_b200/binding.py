@@ -39,6 +39,7 @@ EXPORTS = (
     "sparse_indexer_topk", "compressed_window_attention", "ckv_status_str", "ckv_launch_count",
     "ckv_profile_events", "sparse_indexer_topk_noalloc", "ckv_decode_step_workspace_bytes",
     "ckv_decode_step", "kv_index_append", "ckv_mh_indexer_workspace_bytes", "sparse_mh_indexer_topk",
+    "kv_window_replay",
 )
 CKV_PROF_SCORE, CKV_PROF_ATTENTION = 0, 1
 
@@ -104,6 +105,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ckv_attention_workspace_bytes.restype = sz
     lib.kv_compress_append.argtypes = [P(LayerCfgC), P(LayerCacheC), i32, vp, vp, i32, i32, vp,
                                        vp, vp, vp]
+    lib.kv_window_replay.argtypes = [P(LayerCfgC), P(LayerCacheC), i32, vp, i32, vp, vp, vp, vp]
+    lib.kv_window_replay.restype = ctypes.c_int
     lib.sparse_indexer_topk.argtypes = [P(LayerCfgC), P(LayerCacheC), i32, vp, i32, vp, i32, vp,
                                         vp, vp, vp, sz, vp, vp]
     lib.compressed_window_attention.argtypes = [P(LayerCfgC), P(LayerCacheC), i32, vp, i32, vp,
@@ -290,6 +293,19 @@ def kv_compress_append(cfg: LayerConfig, cache: LayerCache, prev_len: torch.Tens
         ctypes.byref(cfg.c()), ctypes.byref(cache.c()), batch, _ptr(prev_len), _ptr(cu_new),
         max_new if cu_new is not None else 1, max_seq_len, _ptr(kv_new), _ptr(logit_new),
         _ptr(status), _stream(stream)))
+
+
+def kv_window_replay(cfg: LayerConfig, cache: LayerCache, seq_len: torch.Tensor, kv: torch.Tensor,
+                     logit: torch.Tensor, status: torch.Tensor, max_seq_len: int | None = None,
+                     stream=None) -> None:
+    """SWA bounded replay: kv [batch][W][D] / logit [batch][W] hold the recomputed raw tokens of
+    positions L - min(W, L) .. L - 1 (row i = position L - n_w + i)."""
+    batch = int(seq_len.shape[0])
+    if max_seq_len is None:
+        max_seq_len = int(cache.comp_table.shape[1]) * 256
+    _check("kv_window_replay", load_library().kv_window_replay(
+        ctypes.byref(cfg.c()), ctypes.byref(cache.c()), batch, _ptr(seq_len), max_seq_len, _ptr(kv),
+        _ptr(logit), _ptr(status), _stream(stream)))
 
 
 def sparse_indexer_topk(cfg: LayerConfig, cache: LayerCache, seq_len: torch.Tensor,

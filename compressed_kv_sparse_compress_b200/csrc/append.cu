@@ -496,12 +496,47 @@ __global__ void __launch_bounds__(kAppendThreads) append_decode_kernel(AppendArg
   append_decode_slice(a, blockIdx.x, blockIdx.y, threadIdx.x, 0, sm);
 }
 
+// ---------------------------------------------------------------------------- window replay
+
+// SWA bounded replay (aidevelopers.cz "DeepSeek-V4.1-Flash ve vLLM", section "Proc je obnova
+// sliding-window cache draha": after a prefix-cache hit only the last window is replayed and its
+// dependence on older positions is cut). One CTA per (window token i, request b): the caller's raw
+// token of position L - n_w + i (n_w = min(W, L)) is rotated at that position and written to the
+// window cache; if the position belongs to the unfinished group [floor(L/r) r, L) it also goes
+// to its residue ring slot with its logit. Compressed entries are not touched. kv_new rows are
+// [batch][W][D] (row i of request b), logit_new [batch][W]; prev_len holds L.
+__global__ void __launch_bounds__(kAppendThreads) window_replay_kernel(AppendArgs a) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ float red[32];
+  const LayerParams& p = a.p;
+  const int i = blockIdx.x, b = blockIdx.y;
+  const int64_t L = a.prev_len[b];
+  if (L < 1 || L > a.max_seq_len) {
+    if (i == 0 && threadIdx.x == 0) atomicOr(a.status, CKV_DEV_BAD_LENGTH);
+    return;
+  }
+  const int64_t n_w = min(static_cast<int64_t>(p.W), L);
+  if (i >= n_w) return;
+  const int64_t pos = L - n_w + i;
+  const float* raw = a.kv_new + (static_cast<int64_t>(b) * p.W + i) * p.D;
+  const int npairs = p.D / 2;
+  float2 x[kMaxPairsPerThread];
+  for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) x[k] = rotate_raw_pair(a, raw, pr, pos);
+  write_window_token(a, win_row(p, b, pos, a.status), x, red);
+  if (pos >= (L / p.r) * p.r) {
+    float* dst = p.res_kv + (static_cast<int64_t>(b) * p.r + pos % p.r) * p.D;
+    for (int k = 0, pr = threadIdx.x; pr < npairs; ++k, pr += blockDim.x) reinterpret_cast<float2*>(dst)[pr] = x[k];
+    if (threadIdx.x == 0) p.res_logit[static_cast<int64_t>(b) * p.r + pos % p.r] = a.logit_new[static_cast<int64_t>(b) * p.W + i];
+  }
+}
+
 // ---------------------------------------------------------------------------- fused step front
 
 // First kernel of a fused decode step: the append of one slice (threads 0..255) and, on the other
-// 256 threads, the query pass of the same step (q_bar plus the attention's query preparation on
-// sparse layers, the query preparation alone on dense ones), which reads only the query. The two
-// halves synchronise on barriers 1 and 2 and never wait for each other.
+// 256 threads, the query pass of the same step (q_bar and the cos/sin table of the rotary pairs on
+// sparse layers, the table alone on dense ones), which reads only the query. The two halves
+// synchronise on barriers 1 and 2 and never wait for each other.
 template <bool kSparse>
 __global__ void __launch_bounds__(2 * kAppendThreads, 1) step_front_kernel(
     AppendArgs a, int app_slices, const float* q, IndexerWs iws, QueryPrepOut prep, AttnWs aws,
@@ -509,7 +544,7 @@ __global__ void __launch_bounds__(2 * kAppendThreads, 1) step_front_kernel(
   griddep_wait();
   griddep_launch();
   __shared__ AppendDecodeSmem sm;
-  __shared__ double qsm[1024];  // q_bar partial sums [256][2] or the cos/sin table [512][2]
+  __shared__ double qsm[512];  // q_bar partial sums [256][2]
   const int x = blockIdx.x, b = blockIdx.y;
   if (threadIdx.x < kAppendThreads) {
     if (x < app_slices) append_decode_slice(a, x, b, threadIdx.x, 1, sm);
@@ -518,7 +553,7 @@ __global__ void __launch_bounds__(2 * kAppendThreads, 1) step_front_kernel(
       qbar_slice(a.p, a.prev_len, a.max_seq_len, q, iws, a.status, prep, x, b, threadIdx.x - kAppendThreads,
                  reinterpret_cast<double(*)[2]>(qsm), 2);
   } else if (x < prep_parts) {
-    prep_part(a.p, a.prev_len, a.max_seq_len, q, aws, x, b, threadIdx.x - kAppendThreads, qsm, 2);
+    prep_part(a.p, a.prev_len, a.max_seq_len, aws, x, b, threadIdx.x - kAppendThreads);
   }
 }
 
@@ -531,7 +566,7 @@ cudaError_t launch_step_front(const LayerParams& p, int batch, const int32_t* se
   // the new token of request b is at position seq_len[b] - 1
   const AppendArgs a{p, seq_len, nullptr, max_seq_len, kv_new, logit_new, status, -1};
   const int app_slices = p.D / 2 < kSlicePairs ? 1 : p.D / 2 / kSlicePairs;
-  const int prep_parts = attention_tc_supported(p) ? 8 : 1;
+  const int prep_parts = 1;
   const int other = sparse ? kQbarSlices : prep_parts;
   const dim3 grid(app_slices > other ? app_slices : other, batch);
   if (sparse)
@@ -554,6 +589,13 @@ cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_l
   const int gx = static_cast<int>(groups < 512 ? groups : 512);
   dim3 grid(gx, batch);
   return launch_kernel(append_kernel, grid, dim3(kAppendThreads), 0, stream, a);
+}
+
+cudaError_t launch_window_replay(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
+                                 const float* kv, const float* logit, uint32_t* status, cudaStream_t stream) {
+  if (p.W < 1) return cudaSuccess;
+  AppendArgs a{p, seq_len, nullptr, max_seq_len, kv, logit, status, 0};
+  return launch_kernel(window_replay_kernel, dim3(p.W, batch), dim3(kAppendThreads), 0, stream, a);
 }
 
 }  // namespace ckv

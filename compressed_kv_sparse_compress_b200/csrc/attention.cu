@@ -164,8 +164,7 @@ __global__ void __launch_bounds__(kPrepThreads) attn_prep_kernel(LayerParams p, 
                                                                  AttnWs ws) {
   griddep_wait();
   griddep_launch();
-  __shared__ double rope_s[2 * 512];
-  prep_part(p, seq_len, max_seq_len, q, ws, blockIdx.x, blockIdx.y, threadIdx.x, rope_s, 0);
+  prep_part(p, seq_len, max_seq_len, ws, blockIdx.x, blockIdx.y, threadIdx.x);
 }
 
 // Merge of the splits of one (request, head) and inverse rotation for the CUDA-core path (fp32
@@ -285,7 +284,7 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u) {
   return __half22float2(__half2(hr));
 }
 
-// Merge for the tensor-core path (H = 64, D = 512, fp16 partials O_s / c_s): one CTA per
+// Merge for the tensor-core path (H = 64, D = 512, fp16 partials O_s / c_s, maxima in base 2): one CTA per
 // (request, group of kGH heads). Each split's partial rows of the group are 4 KB of contiguous
 // memory; up to kGS splits per round are bulk-copied into shared memory while the block reduces
 // their (m, l) per head, and thread t then merges dims 8 (t % 64) .. 8 (t % 64) + 7 of head
@@ -352,8 +351,8 @@ __global__ void __launch_bounds__(kGThreads, 1) attn_combine_tc_kernel(
     __syncthreads();
     const float Mn = fmaxf(M, fmaxf(red[0][2 * hh], red[0][2 * hh + 1]));
     float w = 0.f, zl = 0.f;
-    if (live) {
-      w = expf(v.x - Mn);
+    if (live) {  // the tensor-core splits keep their maxima in base 2
+      w = exp2f(v.x - Mn);
       zl = w * v.y;
       w *= scv;
     }
@@ -361,7 +360,7 @@ __global__ void __launch_bounds__(kGThreads, 1) attn_combine_tc_kernel(
     zl = warp_sum(zl);
     if (lane == 0) red[1][warp] = zl;
     __syncthreads();
-    const float f = M == -INFINITY ? 0.f : expf(M - Mn);
+    const float f = M == -INFINITY ? 0.f : exp2f(M - Mn);
     Z = Z * f + (red[1][2 * hh] + red[1][2 * hh + 1]);
 #pragma unroll
     for (int k = 0; k < 8; ++k) acc[k] *= f;
@@ -389,7 +388,11 @@ __global__ void __launch_bounds__(kGThreads, 1) attn_combine_tc_kernel(
     o[0] = o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     return;
   }
-  const float inv = Z > 0.f ? 1.f / Z : 0.f;
+  if (!(Z > 0.f)) {  // no key: a zero output (the rotary table may not have been written)
+    o[0] = o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const float inv = 1.f / Z;
   float v8[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) v8[k] = acc[k] * inv;
@@ -438,7 +441,6 @@ AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_
   const size_t ml_bytes = align_up(n_slot * 2 * sizeof(float), 256);
   const size_t sc_bytes = align_up(n_slot * sizeof(float), 256);
   const size_t rope_bytes = align_up(static_cast<size_t>(batch) * (p.d_r / 2 + 1) * 2 * sizeof(double), 256);
-  const size_t q_bytes = attention_tc_supported(p) ? static_cast<size_t>(batch) * kQImageBytes : 0;
   w.half_parts = attention_tc_supported(p);
   if (base) {
     char* c = static_cast<char*>(base);
@@ -446,10 +448,9 @@ AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_
     w.part_h = reinterpret_cast<uint16_t*>(c);
     w.part_ml = reinterpret_cast<float*>(c + o_bytes);
     w.rope = reinterpret_cast<double*>(c + o_bytes + ml_bytes);
-    w.qimage = q_bytes ? reinterpret_cast<uint8_t*>(c + o_bytes + ml_bytes + rope_bytes) : nullptr;
-    w.part_sc = reinterpret_cast<float*>(c + o_bytes + ml_bytes + rope_bytes + q_bytes);
+    w.part_sc = reinterpret_cast<float*>(c + o_bytes + ml_bytes + rope_bytes);
   }
-  w.bytes = o_bytes + ml_bytes + rope_bytes + q_bytes + sc_bytes;
+  w.bytes = o_bytes + ml_bytes + rope_bytes + sc_bytes;
   return w;
 }
 
@@ -458,9 +459,8 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
                              const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
                              uint32_t* status, cudaStream_t stream, bool prep_done) {
   cudaError_t e = cudaSuccess;
-  if (!prep_done) {
-    const dim3 prep_grid(attention_tc_supported(p) ? 8 : 1, batch);   // 8 heads per CTA on the MMA path
-    e = launch_kernel(attn_prep_kernel, prep_grid, dim3(kPrepThreads), 0, stream, p, seq_len, max_seq_len,
+  if (!prep_done && !attention_tc_supported(p)) {  // the tensor-core kernel writes the table itself
+    e = launch_kernel(attn_prep_kernel, dim3(1, batch), dim3(kPrepThreads), 0, stream, p, seq_len, max_seq_len,
                       q, ws);
     if (e != cudaSuccess) return e;
   }

@@ -1,29 +1,47 @@
 // Tensor-core attention path (tcgen05, kind::f16, fp32 accumulation in tensor memory) for
-// H = 64 query heads sharing one K=V vector of D = 512 (multi-query attention).
+// H = 64 query heads sharing one K=V vector of D = 512 (multi-query attention), over a bf16 or
+// NVFP4 compressed cache and an FP8 window.
 //
 // 24-ai.news "vLLM uveo DeepSeek V4 s 8,7x manjim KV cacheom", section "Kako funkcionira
 // optimizacija KV cachea?": every head reads the same shared K=V vector, so the heads x keys
 // contractions are dense matrix products; aidevelopers.cz "DeepSeek-V4.1-Flash ve vLLM", section
 // "Vykon neprinesl jeden kernel": attention over an NVFP4 compressed cache.
 //
-// Orientation: keys are the MMA's M dimension (128 keys per tile) and heads its N dimension (64),
-// so every MMA runs at M = 128:
-//     S^T[keys, heads]  = X[keys, D]  . Q~^T[D, heads]        A = X   (K-major), B = Q~ (K-major)
-//     O^T[D, heads]    += X^T[D, keys] . P^T[keys, heads]     A = X^T (MN-major), B = P (MN-major)
-// One fp16 copy of the key tile X in shared memory (128-byte swizzled rows of 64 elements) is the
-// K-major A operand of the first product and the MN-major A operand of the second. The cache is
-// converted to fp16 while it is staged: bf16 and e2m1 x e4m3 values are exact in fp16 (|x| <
-// 65504), FP8 window codes are exact and their per-token scale is applied to the logits and to
-// P in fp32. Q~ (rotated query) is rounded to fp16 once. S^T (64 columns) and O^T (4 blocks of 64
-// columns) live in tensor memory. The CTA has 32 warps, so that the gather of a tile's key rows
-// has many loads in flight; for the softmax warp w owns the keys of TMEM lane quarter w%4 (one
-// key per thread) and 8 heads; per-head maxima and sums are reduced across the keys with warp
-// reduce-scatters. The running maximum is only raised when a tile's maximum exceeds it by more
-// than 8 (then O^T is rescaled in tensor memory), so P <= e^8 stays well inside fp16.
+// Products (keys in tiles of 32; all operands fp16 in shared memory, 128-byte swizzled rows):
+//     S[hi|lo, keys]  = [Q'hi; Q'lo] . X'^T     M = 128 (the 64 hi rows of the query, then its 64
+//                                               lo rows), N = 32 keys, K = D; A = Q', B = X'
+//                                               (both K-major)
+//     O^T[D, heads]  += X'^T . P^T               M = 128 dims (4 blocks), N = 64 heads, K = keys;
+//                                               A = X'^T (MN-major: the same tile), B = P (K-major)
+// Exactness: the rotated query of head h is scaled by a power of two g_h^-1 (its largest element
+// lands in [2^8, 2^9)) and split into fp16 hi + lo parts, which carry its fp32 value to about
+// 2^-22; each key is scaled by a power of two of its own (largest element in [2^8, 2^9)) before
+// it is converted to fp16, which is exact for bf16 values, e4m3 codes and e2m1 x e4m3 products
+// whatever their magnitude. The logit of (head h, key j) is (S_hi + S_lo) g_h f_j sm_scale
+// log2(e), where the value factor f_j is the key's power of two times its FP8 token scale (1 for
+// the compressed entries). The softmax runs in base 2 with a running maximum that is raised only
+// when a tile exceeds it by more than 8 nats; the weights enter P as p_j f_j / F, F being a
+// power-of-two running bound of the value factors raised only past 16 F, so P stays below 2^16
+// and O^T = F^-1 sum_j p_j x_j. Raising either bound rescales O^T in tensor memory.
 //
-// Each CTA handles `tiles_per_split` consecutive tiles of one request's key list and writes the
-// same un-normalised partials (max, sum, output) as the CUDA-core path; the shared combine kernel
-// merges the splits and applies the inverse rotation.
+// Warp roles (672 threads):
+//   warps 0..3   softmax: warp w reads TMEM lane quarter w (w < 2: the hi rows of heads
+//                32w .. 32w+31; w >= 2: their lo rows); a hi warp and its lo partner swap half of
+//                their keys through shared memory, so that each thread owns 16 keys of one head
+//   warp 4       owns the tensor memory; lane 0 issues every MMA (the logits of tile t+1 before
+//                the output product of tile t, so the tensor pipe works while the softmax runs)
+//   warps 5..20  loaders: each resolves the pool rows of its 2 keys of every tile, keeps the raw
+//                bytes of the next two tiles in flight in registers and converts a tile into the
+//                fp16 operand image once its shared-memory stage (one of 2) is free; they also
+//                build the query image at the start and write the partial outputs at the end
+// Every wait on an mbarrier is bounded; a role that gives up raises an abort flag that the others
+// poll, every issued MMA is drained before the epilogue and before the tensor memory is freed, and
+// the split is then marked empty with CKV_DEV_TIMEOUT set.
+//
+// Each CTA takes keys_per_split consecutive keys of one request's key list (the window tokens
+// [max(0, L-W), L) first, then the selected entries, or every entry of a dense layer) and writes
+// an un-normalised partial (maximum in base 2, sum, output rows as fp16 with a power-of-two
+// scale); the combine kernel merges the splits and applies the inverse rotation.
 
 #include "ckv_internal.h"
 #include "ckv_ptx.cuh"
@@ -33,38 +51,55 @@ namespace {
 
 constexpr int kH = 64;
 constexpr int kD = 512;
-constexpr int kTile = 128;
-constexpr int kThreads = 1024;  // 32 warps: many loads in flight per SM while staging
-constexpr int kChunks = kD / 64;
-constexpr uint32_t kXChunk = kTile * 128;        // bytes of one 64-element chunk of the tile
-constexpr uint32_t kXBytes = kXChunk * kChunks;  // 128 KB
-constexpr uint32_t kQChunk = kH * 128;
-constexpr uint32_t kQBytes = kQChunk * kChunks;  // 64 KB
-constexpr uint32_t kPBytes = kTile * kH * 2;     // 16 KB
-constexpr uint32_t kSCol = 0;
-constexpr uint32_t kOCol = 256;
+constexpr int kTile = 32;                              // keys per tile (N of the logits product)
+constexpr int kMaxTiles = 16;                          // tiles per split at most
+constexpr int kChunks = kD / 64;                       // 64-dim chunks (128-byte rows)
+constexpr int kSoftWarps = 4;
+constexpr int kMmaWarp = 4;
+constexpr int kFirstLoadWarp = 5;
+constexpr int kLoadWarps = 16;
+constexpr int kThreads = 32 * (kFirstLoadWarp + kLoadWarps);  // 672
+constexpr int kLoadThreads = 32 * kLoadWarps;
+constexpr int kSoftThreads = 32 * kSoftWarps;
+static_assert(kTile == 2 * kLoadWarps, "each loader warp stages two keys of a tile");
+static_assert(kMaxTiles * 2 <= 32, "one lane of a loader warp per (tile, key) of the split");
+static_assert(kH == 4 * kLoadWarps, "each loader warp builds the query image of four heads");
+
+constexpr uint32_t kQChunk = 2 * kH * 128;             // 16 KB: 64 hi rows, then 64 lo rows
+constexpr uint32_t kQBytes = kQChunk * kChunks;        // 128 KB
+constexpr uint32_t kXChunk = kTile * 128;              // 4 KB
+constexpr uint32_t kXStage = kXChunk * kChunks;        // 32 KB
+constexpr uint32_t kPBytes = kH * 128;                 // 8 KB: row = head; stage s in bytes 64s..64s+63
+constexpr uint32_t kXchStride = 20;                    // floats per lane in an exchange slot
+constexpr uint32_t kXchSlot = 32 * kXchStride * 4;     // 2560 B
+constexpr uint32_t kSCol = 0;                          // S stage s: columns 32 s
+constexpr uint32_t kOCol = 256;                        // O^T dims block m: columns 256 + 64 m
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescale = 8.0f;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRaiseLog2 = 8.0f * kLog2e;            // the running max moves past +8 nats
+constexpr float kRaiseF = 16.0f;                       // the value bound moves past 16x
 
 // shared memory carve-up (byte offsets from a 1024-aligned base)
-constexpr uint32_t kOffX = 0;
-constexpr uint32_t kOffQ = kOffX + kXBytes;
-constexpr uint32_t kOffP = kOffQ + kQBytes;          // also the rotary table in the prologue
-constexpr uint32_t kOffRow = kOffP + kPBytes;        // int64[128] pool row (-1: absent key)
-constexpr uint32_t kOffLs = kOffRow + 8 * kTile;     // float[128] logit factor per key
-constexpr uint32_t kOffVs = kOffLs + 4 * kTile;      // float[128] value factor per key
-constexpr uint32_t kOffWin = kOffVs + 4 * kTile;     // int[128]   1: window token
-constexpr uint32_t kOffRed = kOffWin + 4 * kTile;    // float[4][64]
-constexpr uint32_t kOffM = kOffRed + 4 * 4 * kH;     // float[64] running max
-constexpr uint32_t kOffA = kOffM + 4 * kH;           // float[64] rescale factor of this tile
-constexpr uint32_t kOffL = kOffA + 4 * kH;           // float[64] running sum
-constexpr uint32_t kOffFlag = kOffL + 4 * kH;        // int[4]
-constexpr uint32_t kOffBar = kOffFlag + 16;          // uint64 mbarrier: MMA completion
-constexpr uint32_t kOffBarQ = kOffBar + 8;           // uint64 mbarrier: query bytes landed
-constexpr uint32_t kOffTmem = kOffBarQ + 8;          // uint32 TMEM base
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffX = kOffQ + kQBytes;
+constexpr uint32_t kOffP = kOffX + 2 * kXStage;
+constexpr uint32_t kOffXch = kOffP + kPBytes;            // float[4 slots][32 lanes][20]
+constexpr uint32_t kOffKf = kOffXch + 4 * kXchSlot;      // float[2 stages][32]: key value factors
+constexpr uint32_t kOffRed = kOffKf + 2 * kTile * 4;     // float[2][4][32]: max and bound per lane
+constexpr uint32_t kOffAlpha = kOffRed + 2 * 4 * 32 * 4; // float[64]: O^T rescale per head
+constexpr uint32_t kOffQs = kOffAlpha + kH * 4;          // float[64]: query scale g_h per head
+constexpr uint32_t kOffEpi = kOffQs + kH * 4;            // float[4][64]: output amax per lane quarter
+constexpr uint32_t kOffMisc = kOffEpi + 4 * kH * 4;      // int abort; float F
+constexpr uint32_t kOffBar = kOffMisc + 16;              // 11 mbarriers
+constexpr uint32_t kOffTmem = kOffBar + 11 * 8;
 constexpr uint32_t kSmemUsed = kOffTmem + 8;
 constexpr int kSmemBytes = static_cast<int>(kSmemUsed) + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+// mbarriers: xfull[2] (loaders -> MMA, softmax), xfree[2] (output product of the stage's tile
+// done -> loaders, softmax), sfull[2] (logits done -> softmax), sfree[2] (softmax read the logits
+// -> MMA), pfull[2] (softmax wrote P -> MMA), drain (every MMA done)
+constexpr int kBarXfull = 0, kBarXfree = 2, kBarSfull = 4, kBarSfree = 6, kBarPfull = 8, kBarDrain = 10;
 
 // ------------------------------------------------------------------------------------ PTX
 
@@ -120,9 +155,10 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   return d;
 }
 
-// instruction descriptor, kind::f16: fp32 accumulator, fp16 A and B, M = 128, N = 64
-constexpr uint32_t kIdescS = (1u << 4) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescPV = kIdescS | (1u << 15) | (1u << 16);  // A and B MN-major
+// instruction descriptors, kind::f16 with fp32 accumulation and fp16 A and B:
+//   logits: M = 128, N = 32, A and B K-major;  output: M = 128, N = 64, A MN-major, B K-major
+constexpr uint32_t kIdescS = (1u << 4) | ((32u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | ((64u >> 3) << 17) | ((128u >> 4) << 24) | (1u << 15);
 
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n"
@@ -138,6 +174,48 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// barrier `id` over `n` threads that also ANDs (kAnd) or ORs a predicate across them
+template <bool kAnd>
+__device__ __forceinline__ bool bar_red(int id, int n, bool v) {
+  uint32_t out;
+  if constexpr (kAnd) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %1, 0;\n bar.red.and.pred p, %2, %3, p;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(out)
+        : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %1, 0;\n bar.red.or.pred p, %2, %3, p;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(out)
+        : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+        : "memory");
+  }
+  return out != 0;
+}
+
+// bounded wait for the completion of the barrier phase with parity `phase`; also gives up once
+// another role has raised the abort flag
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t phase, volatile int* abort_flag) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_try_wait(bar, phase)) return true;
+    if ((i & 255u) == 255u && *abort_flag) return false;
+  }
+  return false;
+}
+
 // ------------------------------------------------------------------------------------ helpers
 
 __device__ __forceinline__ uint32_t half2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
@@ -146,450 +224,576 @@ __device__ __forceinline__ uint32_t pack_f32x2(float a, float b) {
   return half2_bits(__floats2half2_rn(a, b));
 }
 
-__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
-  __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
-  return half2_bits(__half2(r));
+// 2^e as a float for -126 <= e <= 127
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// the power-of-two shift that puts a largest magnitude with float bits `mb` into [2^8, 2^9)
+// (0 for an all-zero vector), within the range where both 2^shift and 2^-shift are normal
+__device__ __forceinline__ int norm_shift(uint32_t mb) {
+  if (mb == 0u) return 0;
+  const int e = static_cast<int>(mb >> 23) - 127;
+  return max(-126, min(126, 8 - e));
 }
 
-// Reduction of N (64 or 32) per-thread values across a warp; afterwards t[0 .. N/32) hold the
-// reduction of entries (N/32)*lane .. (N/32)*lane + N/32 - 1.
-template <int N, bool kMax>
-__device__ __forceinline__ void reduce_scatter(float (&t)[N], int lane) {
-#pragma unroll
-  for (int s = 0; s < 5; ++s) {
-    const int o = 16 >> s;
-    const int half = N >> (s + 1);
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = upper ? t[i] : t[i + half];
-      const float keep = upper ? t[i + half] : t[i];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, o);
-      t[i] = kMax ? fmaxf(keep, recv) : keep + recv;
-    }
-  }
+// the smallest power of two >= x (x finite and > 0)
+__device__ __forceinline__ float pow2_ceil(float x) {
+  const uint32_t u = __float_as_uint(x);
+  const uint32_t e = (u >> 23) + ((u & 0x7fffffu) != 0u ? 1u : 0u);
+  return e >= 255u ? INFINITY : __uint_as_float(e << 23);
 }
 
-// Reduction of one value per (head of 8, lane) over the warp's 32 lanes: three reduce-scatter
-// stages, then two butterfly stages; lane l returns the reduction of entry l >> 2.
-template <bool kMax>
-__device__ __forceinline__ float warp_reduce8(float (&t)[8], int lane) {
-  reduce_scatter<8, kMax>(t, lane);
-  float v = t[0];
-#pragma unroll
-  for (int o = 2; o > 0; o >>= 1) {
-    const float x = __shfl_xor_sync(0xffffffffu, v, o);
-    v = kMax ? fmaxf(v, x) : v + x;
-  }
-  return v;
-}
-
-// raw bytes of one 8-element granule of a key, loaded before conversion
+// Raw bytes of one 8-element granule of a key: bf16 16 B, FP8 window 8 B, NVFP4 4 B of codes and
+// the e4m3 scale of its 16-element block.
 struct Raw {
-  uint4 a, b;
+  uint4 a;
   uint32_t s;
 };
 
-template <int CT, int WT>
+template <int CT>
 __device__ __forceinline__ Raw load_granule(const LayerParams& p, int64_t row, bool win, int g) {
   Raw r;
   r.a = make_uint4(0, 0, 0, 0);
-  r.b = make_uint4(0, 0, 0, 0);
   r.s = 0;
   if (row < 0) return r;
   if (win) {
-    const uint8_t* base = p.win_codes + row * p.win_row_bytes;
-    if constexpr (WT == CKV_FP8_E4M3) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(base) + g);
-      r.a.x = v.x;
-      r.a.y = v.y;
-    } else {
-      r.a = __ldg(reinterpret_cast<const uint4*>(base) + 2 * g);
-      r.b = __ldg(reinterpret_cast<const uint4*>(base) + 2 * g + 1);
-    }
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.win_codes + row * p.win_row_bytes) + g);
+    r.a.x = v.x;
+    r.a.y = v.y;
     return r;
   }
   const uint8_t* base = p.comp_codes + row * p.comp_row_bytes;
   if constexpr (CT == CKV_BF16) {
     r.a = __ldg(reinterpret_cast<const uint4*>(base) + g);
-  } else if constexpr (CT == CKV_NVFP4) {
+  } else {
     r.a.x = __ldg(reinterpret_cast<const uint32_t*>(base) + g);
     r.s = __ldg(p.comp_scales + row * (kD / 16) + (g >> 1));
-  } else {
-    r.a = __ldg(reinterpret_cast<const uint4*>(base) + 2 * g);
-    r.b = __ldg(reinterpret_cast<const uint4*>(base) + 2 * g + 1);
   }
   return r;
 }
 
-template <int CT, int WT>
-__device__ __forceinline__ uint4 convert_granule(const Raw& r, bool win) {
+// the granule's 8 values as fp32 (exact): e4m3 codes of a window token (its scale is applied
+// through the key factor), bf16 values, or e2m1 codes times their block's e4m3 scale
+template <int CT>
+__device__ __forceinline__ void decode_granule(const Raw& r, bool win, float (&v)[8]) {
   if (win) {
-    if constexpr (WT == CKV_FP8_E4M3) {
-      return make_uint4(e4m3x2_to_h2(r.a.x), e4m3x2_to_h2(r.a.x >> 16), e4m3x2_to_h2(r.a.y),
-                        e4m3x2_to_h2(r.a.y >> 16));
-    } else {
-      return make_uint4(pack_f32x2(__uint_as_float(r.a.x), __uint_as_float(r.a.y)),
-                        pack_f32x2(__uint_as_float(r.a.z), __uint_as_float(r.a.w)),
-                        pack_f32x2(__uint_as_float(r.b.x), __uint_as_float(r.b.y)),
-                        pack_f32x2(__uint_as_float(r.b.z), __uint_as_float(r.b.w)));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w = i < 2 ? r.a.x : r.a.y;
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((w >> (16 * (i & 1))) & 0xffffu), __NV_E4M3);
+      const float2 f = __half22float2(__half2(h));
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
     }
+    return;
   }
   if constexpr (CT == CKV_BF16) {
     const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
-    uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = pack_f32x2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
-    return make_uint4(o[0], o[1], o[2], o[3]);
-  } else if constexpr (CT == CKV_NVFP4) {
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  } else {
     const __half s = __half(__nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(r.s), __NV_E4M3));
     const __half2 s2 = __half2(s, s);
-    uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = half2_bits(__hmul2(e2m1x2_to_half2(static_cast<uint8_t>(r.a.x >> (8 * i))), s2));
-    return make_uint4(o[0], o[1], o[2], o[3]);
-  } else {
-    return make_uint4(pack_f32x2(__uint_as_float(r.a.x), __uint_as_float(r.a.y)),
-                      pack_f32x2(__uint_as_float(r.a.z), __uint_as_float(r.a.w)),
-                      pack_f32x2(__uint_as_float(r.b.x), __uint_as_float(r.b.y)),
-                      pack_f32x2(__uint_as_float(r.b.z), __uint_as_float(r.b.w)));
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(__hmul2(e2m1x2_to_half2(static_cast<uint8_t>(r.a.x >> (8 * i))), s2));
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
   }
 }
 
-// byte offset of 16-byte granule g of row `row` in a 128-byte-swizzled operand made of chunks
-// of `chunk_bytes` (64 elements per row and chunk)
+// byte offset of 16-byte granule g (8 dims) of row `row` in an operand made of 64-dim chunks of
+// `chunk_bytes`, rows of 128 bytes with the 128-byte swizzle
 __device__ __forceinline__ uint32_t swz(uint32_t chunk_bytes, int row, int g) {
   return static_cast<uint32_t>(g >> 3) * chunk_bytes + static_cast<uint32_t>(row) * 128u +
          (static_cast<uint32_t>((g & 7) ^ (row & 7)) << 4);
 }
 
-// Pool row, window flag and factors of the keys of one tile (threads 0..127, one key each):
-// the logit factor is sm_scale times the window token's FP8 scale, the value factor that scale.
-template <int WT>
-__device__ __forceinline__ void key_meta(const LayerParams& p, int b, int L, const int32_t* idx,
-                                         int idx_stride, int64_t n_c, int64_t n_sel, int64_t n_win,
-                                         int64_t k_first, int64_t k_end, int64_t* key_row,
-                                         int* key_win, float* key_vs, float* key_ls,
-                                         uint32_t* status) {
-  const int tid = threadIdx.x;
-  if (tid >= kTile) return;
-  const int64_t kk = k_first + tid;
-  int64_t row = -1;
-  int win = 0;
-  float vs = 1.f;
-  if (kk < k_end) {
-    if (kk < n_sel) {
-      const int64_t ent = idx ? idx[static_cast<int64_t>(b) * idx_stride + kk] : kk;
-      if (ent < 0 || ent >= n_c) atomicOr(status, CKV_DEV_BAD_INDEX);
-      else row = comp_row(p, b, ent, status);
-    } else {
-      win = 1;
-      row = win_row(p, b, L - n_win + (kk - n_sel), status);
-      if (row >= 0 && WT == CKV_FP8_E4M3) vs = p.win_scales[row];
-    }
+// The key list of request b: window tokens first, then the selected (or all) entries.
+struct Keys {
+  int L;
+  int64_t n_c, n_sel, n_win, n_keys;
+};
+
+// Pool row (-1: absent, with the status bit set) of key k of request b; window keys set *win.
+__device__ __forceinline__ int64_t key_row(const LayerParams& p, const Keys& kl, int b, const int32_t* idx,
+                                           int idx_stride, int64_t k, bool* win, uint32_t* status) {
+  *win = k < kl.n_win;
+  if (*win) return win_row(p, b, kl.L - kl.n_win + k, status);
+  const int64_t e = k - kl.n_win;
+  const int64_t ent = idx ? idx[static_cast<int64_t>(b) * idx_stride + e] : e;
+  if (ent < 0 || ent >= kl.n_c) {
+    atomicOr(status, CKV_DEV_BAD_INDEX);
+    return -1;
   }
-  key_row[tid] = row;
-  key_win[tid] = win;
-  key_vs[tid] = vs;
-  key_ls[tid] = p.sm_scale * vs;
+  return comp_row(p, b, ent, status);
 }
 
 // ------------------------------------------------------------------------------------ kernel
 
-template <int CT, int WT>
+template <int CT>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const float* q, const int32_t* idx,
     const int32_t* cnt, int idx_stride, AttnWs ws, uint32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(base);
-  int64_t* key_row = reinterpret_cast<int64_t*>(base + kOffRow);
-  float* key_ls = reinterpret_cast<float*>(base + kOffLs);
-  float* key_vs = reinterpret_cast<float*>(base + kOffVs);
-  int* key_win = reinterpret_cast<int*>(base + kOffWin);
+  float* kf = reinterpret_cast<float*>(base + kOffKf);
   float* red = reinterpret_cast<float*>(base + kOffRed);
-  float* m_run = reinterpret_cast<float*>(base + kOffM);
-  float* alpha = reinterpret_cast<float*>(base + kOffA);
-  float* l_run = reinterpret_cast<float*>(base + kOffL);
-  int* flags = reinterpret_cast<int*>(base + kOffFlag);
-  const uint32_t bar = sb + kOffBar;
+  float* alpha_sm = reinterpret_cast<float*>(base + kOffAlpha);
+  float* qs = reinterpret_cast<float*>(base + kOffQs);
+  float* epi = reinterpret_cast<float*>(base + kOffEpi);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc);
+  float* f_final = reinterpret_cast<float*>(base + kOffMisc + 4);
+  auto bar = [&](int i) { return sb + kOffBar + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffTmem);
 
   const int b = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t bar_q = sb + kOffBarQ;
 
-  // ---- set-up that reads no global memory, before waiting for the previous kernel: barriers,
-  //      running max and sum, tensor memory
+  // ---- set-up that reads no global memory, before waiting for the previous kernel
   if (tid == 0) {
-    mbar_init(bar, 1);
-    mbar_init(bar_q, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarXfull + s), kLoadWarps);
+      mbar_init(bar(kBarXfree + s), 1);
+      mbar_init(bar(kBarSfull + s), 1);
+      mbar_init(bar(kBarSfree + s), kSoftThreads);
+      mbar_init(bar(kBarPfull + s), kSoftThreads);
+    }
+    mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    *f_final = 0.f;
     fence_proxy_async();
-    flags[0] = flags[1] = 0;
   }
-  if (tid < kH) {
-    m_run[tid] = -INFINITY;
-    l_run[tid] = 0.f;
-  }
-  if (warp == 0) tmem_alloc(sb + kOffTmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_alloc(sb + kOffTmem, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  auto release = [&]() {   // every exit after the allocation (block-uniform)
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-      tc_fence_after();
-      tmem_dealloc(tmem, kTmemCols);
-    }
-  };
   griddep_wait();
   griddep_launch();
 
-  const int L = seq_len[b];
-  if (L < 1 || L > max_seq_len) {  // flagged by the combine
-    release();
-    return;
+  Keys kl;
+  kl.L = seq_len[b];
+  const bool live = kl.L >= 1 && kl.L <= max_seq_len;  // a bad length is flagged by the combine
+  kl.n_c = live ? kl.L / p.r : 0;
+  kl.n_sel = !live ? 0 : idx ? min(static_cast<int64_t>(max(cnt[b], 0)), static_cast<int64_t>(idx_stride)) : kl.n_c;
+  kl.n_win = live ? min(p.W, kl.L) : 0;
+  kl.n_keys = kl.n_win + kl.n_sel;
+  // the cos/sin of every rotary pair at the query position, for the combine's inverse rotation
+  if (live && split == 0 && tid < p.d_r / 2) {
+    double sn, cs;
+    sincos(static_cast<double>(kl.L - 1) * rope_inv_freq(p, tid), &sn, &cs);
+    double* rope_g = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
+    rope_g[2 * tid] = cs;
+    rope_g[2 * tid + 1] = sn;
   }
-  const int64_t n_c = L / p.r;
-  const int64_t n_sel = idx ? min(static_cast<int64_t>(max(cnt[b], 0)), static_cast<int64_t>(idx_stride)) : n_c;
-  const int64_t n_win = min(p.W, L);
-  const int64_t n_keys = n_sel + n_win;
   const int64_t k_begin = static_cast<int64_t>(split) * ws.keys_per_split;
-  if (k_begin >= n_keys) {
-    release();
+  if (k_begin >= kl.n_keys) {  // nothing to attend (uniform across the CTA)
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
+    }
     return;
   }
-  const int64_t k_end = min(n_keys, k_begin + ws.keys_per_split);
-  const int n_tiles = static_cast<int>((k_end - k_begin + kTile - 1) / kTile);
+  const int nk = static_cast<int>(min(kl.n_keys - k_begin, static_cast<int64_t>(ws.keys_per_split)));
+  const int n_tiles = (nk + kTile - 1) / kTile;
+  const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
 
-  // ---- the prepared query image (64 KB, written per request by the prep kernel) is bulk-copied
-  //      into the Q region while the keys of tile 0 are resolved and staged
-  if (tid == 0) {
-    const uint8_t* img = ws.qimage + static_cast<int64_t>(b) * kQBytes;
-    constexpr uint32_t kPiece = 16384;
-    mbar_expect_tx(bar_q, kQBytes);
-#pragma unroll 1
-    for (uint32_t off = 0; off < kQBytes; off += kPiece) bulk_g2s(sb + kOffQ + off, img + off, kPiece, bar_q);
-  }
-  key_meta<WT>(p, b, L, idx, idx_stride, n_c, n_sel, n_win, k_begin, k_end, key_row, key_win, key_vs,
-               key_ls, status);
-  __syncthreads();
-  uint32_t phase = 0;
-  bool ok = true;
-  bool q_ready = false;
-
-  for (int tile = 0; tile < n_tiles && ok; ++tile) {
-    const int64_t k_first = k_begin + static_cast<int64_t>(tile) * kTile;
-    const int n_valid = static_cast<int>(min(static_cast<int64_t>(kTile), k_end - k_first));
-    if (tile > 0) {
-      key_meta<WT>(p, b, L, idx, idx_stride, n_c, n_sel, n_win, k_begin + static_cast<int64_t>(tile) * kTile,
-                   k_end, key_row, key_win, key_vs, key_ls, status);
-      __syncthreads();
+  // ---- prologue (loaders): resolve the rows of their keys, put the first two tiles' loads in
+  //      flight, build the query image (4 heads per warp)
+  const int li = warp - kFirstLoadWarp;  // loader index (warps >= kFirstLoadWarp)
+  // lane j of a loader warp holds the row of key 2 li + (j & 1) of tile j >> 1
+  long long my_row = -1;
+  int my_win = 0;
+  float my_tscale = 1.f;
+  Raw ring[2][2][2];  // [tile parity][key u][granule lane, lane + 32]
+  auto row_of = [&](int t, int u, bool* win, float* tsc) -> int64_t {
+    const int src = 2 * t + u;
+    *win = __shfl_sync(0xffffffffu, my_win, src) != 0;
+    *tsc = __shfl_sync(0xffffffffu, my_tscale, src);
+    return static_cast<int64_t>(__shfl_sync(0xffffffffu, my_row, src));
+  };
+  auto issue = [&](int t, Raw (&r)[2][2]) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      bool win;
+      float tsc;
+      const int64_t row = row_of(t, u, &win, &tsc);
+      r[u][0] = load_granule<CT>(p, row, win, lane);
+      r[u][1] = load_granule<CT>(p, row, win, lane + 32);
     }
+  };
+  if (warp >= kFirstLoadWarp) {
+    const int t = lane >> 1, u = lane & 1;
+    const int kloc = t * kTile + 2 * li + u;
+    if (t < n_tiles && kloc < nk) {
+      bool win;
+      my_row = key_row(p, kl, b, idx, idx_stride, k_begin + kloc, &win, status);
+      my_win = win ? 1 : 0;
+      if (win && my_row >= 0) my_tscale = p.win_scales[my_row];
+    }
+    issue(0, ring[0]);
+    if (n_tiles > 1) issue(1, ring[1]);
 
-    // ---- stage the tile as fp16 (absent keys are zero rows): warp w converts kpw consecutive
-    //      keys (4 of a full tile, 2 when it holds at most 64 keys), lane l the granules l and l+32
-    //      of each (the key's row and kind read once per key), all of them in flight at once. Rows
-    //      that are not staged hold stale or uninitialised values: their logits are masked and no
-    //      PV step reads them.
-    {
-      constexpr int kB = (CT == CKV_F32 || WT == CKV_F32) ? 2 : 4;  // fp32 granules are 32 bytes
-      const int kpw = n_valid > kTile / 2 ? 4 : 2;
+    // query image, heads 4 li .. 4 li + 3: lane l holds dims 16 l .. 16 l + 15 (granules 2l,
+    // 2l + 1 of chunk l/4); the rotary pairs 8 l .. 8 l + 7 are rotated at the query position L-1
+    // (fp64 angles); hi rows are h, lo rows 64 + h
+    const int first_rope = (kD - p.d_r) / 2;
+    const float* qb = q + static_cast<int64_t>(b) * kH * kD;
+#pragma unroll 1
+    for (int hh = 0; hh < 4; ++hh) {
+      const int h = 4 * li + hh;
+      float x[16];
 #pragma unroll
-      for (int u0 = 0; u0 < 4; u0 += kB) {
-        if (u0 >= kpw) break;
-        Raw r[kB][2];
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          if (u0 + u < kpw) {
-            const int j = kpw * warp + u0 + u;
-            const int64_t row = key_row[j];
-            const bool win = key_win[j] != 0;
-            r[u][0] = load_granule<CT, WT>(p, row, win, lane);
-            r[u][1] = load_granule<CT, WT>(p, row, win, lane + 32);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          if (u0 + u < kpw) {
-            const int j = kpw * warp + u0 + u;
-            const bool win = key_win[j] != 0;
-            st_shared_v4(sb + kOffX + swz(kXChunk, j, lane), convert_granule<CT, WT>(r[u][0], win));
-            st_shared_v4(sb + kOffX + swz(kXChunk, j, lane + 32), convert_granule<CT, WT>(r[u][1], win));
+      for (int k = 0; k < 4; ++k) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(qb + static_cast<int64_t>(h) * kD + 16 * lane) + k);
+        x[4 * k] = v.x;
+        x[4 * k + 1] = v.y;
+        x[4 * k + 2] = v.z;
+        x[4 * k + 3] = v.w;
+      }
+      if (8 * lane + 7 >= first_rope) {
+#pragma unroll 1
+        for (int k = 0; k < 8; ++k) {
+          const int pr = 8 * lane + k;
+          if (pr >= first_rope) {
+            double rs, rc;
+            sincos(static_cast<double>(kl.L - 1) * rope_inv_freq(p, pr - first_rope), &rs, &rc);
+            const double a0 = x[2 * k], a1 = x[2 * k + 1];
+            x[2 * k] = static_cast<float>(a0 * rc - a1 * rs);
+            x[2 * k + 1] = static_cast<float>(a0 * rs + a1 * rc);
           }
         }
       }
+      uint32_t mb = 0;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) mb = max(mb, __float_as_uint(x[k]) & 0x7fffffffu);
+      const int sh = norm_shift(__reduce_max_sync(0xffffffffu, mb));
+      const float up = exp2i(sh);
+      if (lane == 0) qs[h] = exp2i(-sh);
+      uint32_t hi[8], lo[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float a = x[2 * k] * up, c = x[2 * k + 1] * up;
+        const __half2 h16 = __floats2half2_rn(a, c);
+        const float2 back = __half22float2(h16);
+        hi[k] = half2_bits(h16);
+        lo[k] = pack_f32x2(a - back.x, c - back.y);
+      }
+      const uint32_t qa = sb + kOffQ;
+      st_shared_v4(qa + swz(kQChunk, h, 2 * lane), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+      st_shared_v4(qa + swz(kQChunk, h, 2 * lane + 1), make_uint4(hi[4], hi[5], hi[6], hi[7]));
+      st_shared_v4(qa + swz(kQChunk, kH + h, 2 * lane), make_uint4(lo[0], lo[1], lo[2], lo[3]));
+      st_shared_v4(qa + swz(kQChunk, kH + h, 2 * lane + 1), make_uint4(lo[4], lo[5], lo[6], lo[7]));
     }
     fence_proxy_async();
-    tc_fence_before();
-    if (!q_ready) {   // the query image must have landed before the first MMA reads it
-      ok = __syncthreads_and(mbar_wait(bar_q, 0)) != 0;
-      q_ready = true;
+  }
+  __syncthreads();  // the query image and its scales
+
+  if (warp == kMmaWarp) {
+    if (lane == 0) {
+      // ---------------- MMAs: the logits of tile t, then the output product of tile t-1
+      bool issued = false;
+      auto pv = [&](int u) -> bool {
+        const int s = u & 1;
+        if (!wait_or_abort(bar(kBarPfull + s), static_cast<uint32_t>(u >> 1) & 1u, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t xs = sb + kOffX + s * kXStage;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint64_t bp = sdesc(sb + kOffP + 64 * s + 32 * kk, 16, 1024);
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            mma_f16(tmem + kOCol + 64 * m, sdesc(xs + 2 * m * kXChunk + kk * 2048, kXChunk, 1024), bp, kIdescPV,
+                    (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(kBarXfree + s));
+        return true;
+      };
+      bool ok = true;
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        const int s = t & 1;
+        ok = wait_or_abort(bar(kBarXfull + s), static_cast<uint32_t>(t >> 1) & 1u, abort_flag) &&
+             (t < 2 || wait_or_abort(bar(kBarSfree + s), static_cast<uint32_t>((t >> 1) - 1) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t xs = sb + kOffX + s * kXStage;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16(tmem + kSCol + 32 * s, sdesc(sb + kOffQ + c * kQChunk + ks * 32, 16, 1024),
+                    sdesc(xs + c * kXChunk + ks * 32, 16, 1024), kIdescS, (c | ks) != 0);
+        }
+        mma_commit(bar(kBarSfull + s));
+        issued = true;
+        if (t > 0) ok = pv(t - 1);
+      }
+      if (ok) ok = pv(n_tiles - 1);
+      if (!ok) *abort_flag = 1;
+      if (issued) {  // every MMA issued has completed before O^T is read or the memory freed
+        mma_commit(bar(kBarDrain));
+        if (!mbar_wait(bar(kBarDrain), 0)) *abort_flag = 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp < kSoftWarps) {
+    // ---------------- softmax: thread (quarter q4, lane) = TMEM lane 32 q4 + lane: head h, hi
+    //                  (q4 < 2) or lo rows; after the swap it owns keys kb .. kb + 15 of head h
+    const int q4 = warp;
+    const bool hi_row = q4 < 2;
+    const int h = 32 * (q4 & 1) + lane;
+    const int kb = hi_row ? 0 : 16;
+    const float ch = qs[h] * p.sm_scale * kLog2e;
+    float* xch_mine = reinterpret_cast<float*>(base + kOffXch + q4 * kXchSlot) + lane * kXchStride;
+    const float* xch_peer = reinterpret_cast<const float*>(base + kOffXch + (q4 ^ 2) * kXchSlot) + lane * kXchStride;
+    float* red_m = red;            // [4][32]
+    float* red_f = red + 4 * 32;   // [4][32]
+    float m_run = -INFINITY, F_run = 0.f, l_part = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int s = t & 1;
+      const uint32_t ph = static_cast<uint32_t>(t >> 1) & 1u;
+      bool got = __all_sync(0xffffffffu, wait_or_abort(bar(kBarSfull + s), ph, abort_flag) &&
+                                             wait_or_abort(bar(kBarXfull + s), ph, abort_flag));
+      ok = bar_red<true>(1, kSoftThreads, got);  // one decision for the four warps
       if (!ok) break;
-    }
-    __syncthreads();
-
-    // ---- S^T = X . Q~^T
-    if (tid == 128) {
       tc_fence_after();
+      uint32_t raw[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + kSCol + 32 * s, raw);
+      tc_fence_before();
+      mbar_arrive(bar(kBarSfree + s));
+      // swap: a hi row hands its keys 16..31 to its lo partner, a lo row its keys 0..15
+      float own[16], give[16];
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) {
+      for (int i = 0; i < 16; ++i) {
+        own[i] = __uint_as_float(hi_row ? raw[i] : raw[16 + i]);
+        give[i] = __uint_as_float(hi_row ? raw[16 + i] : raw[i]);
+      }
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t a = sdesc(sb + kOffX + c * kXChunk + ks * 32, 16, 1024);
-          const uint64_t bq = sdesc(sb + kOffQ + c * kQChunk + ks * 32, 16, 1024);
-          mma_f16(tmem + kSCol, a, bq, kIdescS, (c | ks) != 0);
+      for (int i = 0; i < 16; i += 4)
+        *reinterpret_cast<float4*>(xch_mine + i) = make_float4(give[i], give[i + 1], give[i + 2], give[i + 3]);
+      named_sync(1, kSoftThreads);
+      float lg[16];
+      float mx = -INFINITY, fmx = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; i += 4) {
+        const float4 o = *reinterpret_cast<const float4*>(xch_peer + i);
+        const float pv4[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float f = kf[s * kTile + kb + i + k];
+          const float sv = own[i + k] + pv4[k];
+          lg[i + k] = f > 0.f ? sv * f * ch : -INFINITY;
+          mx = fmaxf(mx, lg[i + k]);
+          fmx = fmaxf(fmx, f > 0.f ? f : 0.f);
         }
       }
-      mma_commit(bar);
-    }
-    ok = __syncthreads_and(mbar_wait(bar, phase)) != 0;  // uniform across the CTA
-    phase ^= 1;
-    tc_fence_after();
-    if (!ok) break;
-
-    // ---- softmax over the tile's keys: key j = TMEM lane; warp w reads the lanes of quarter w%4
-    //      and the 8 heads of group w/4
-    {
-      const int q4 = warp & 3, hg = warp >> 2;
-      const int j = q4 * 32 + lane;
-      const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-      uint32_t raw[8];
-      tmem_ld8(tmem + lane_base + kSCol + 8 * hg, raw);
-      const float f = key_ls[j];
-      const bool valid = key_row[j] >= 0;
-      float sv[8], t[8];
+      red_m[q4 * 32 + lane] = mx;
+      red_f[q4 * 32 + lane] = fmx;
+      named_sync(1, kSoftThreads);
+      const float mt = fmaxf(mx, red_m[(q4 ^ 2) * 32 + lane]);
+      const float ft = fmaxf(fmx, red_f[(q4 ^ 2) * 32 + lane]);
+      float m_new = m_run, F_new = F_run;
+      if (mt > -INFINITY && (m_run == -INFINITY || mt > m_run + kRaiseLog2)) m_new = mt;
+      if (ft > 0.f && ft > kRaiseF * F_run) F_new = pow2_ceil(ft);
+      const float a_l = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+      const bool moved = m_new != m_run || F_new != F_run;
+      if (hi_row) alpha_sm[h] = F_run > 0.f ? a_l * (F_run / F_new) : 0.f;
+      const bool rescale = bar_red<false>(1, kSoftThreads, t > 0 && moved);  // alpha visible too
+      float psum = 0.f;
+      uint32_t packed[8];
+      const float inv_F = F_new > 0.f ? 1.f / F_new : 0.f;  // a power of two: exact
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        sv[h] = valid ? __uint_as_float(raw[h]) * f : -INFINITY;
-        t[h] = sv[h];
+      for (int i = 0; i < 16; i += 2) {
+        const float p0 = lg[i] > -INFINITY ? exp2f(lg[i] - m_new) : 0.f;
+        const float p1 = lg[i + 1] > -INFINITY ? exp2f(lg[i + 1] - m_new) : 0.f;
+        psum += p0 + p1;
+        const float f0 = kf[s * kTile + kb + i], f1 = kf[s * kTile + kb + i + 1];
+        packed[i >> 1] = pack_f32x2(p0 * (f0 > 0.f ? f0 : 0.f) * inv_F, p1 * (f1 > 0.f ? f1 : 0.f) * inv_F);
       }
-      const float mx = warp_reduce8<true>(t, lane);
-      if ((lane & 3) == 0) red[q4 * kH + 8 * hg + (lane >> 2)] = mx;
-      __syncthreads();
-      if (tid < kH) {
-        const float mt = fmaxf(fmaxf(red[tid], red[kH + tid]), fmaxf(red[2 * kH + tid], red[3 * kH + tid]));
-        const float mo = m_run[tid];
-        float mn = mo, al = 1.f;
-        if (mt > mo + kRescale || (mo == -INFINITY && mt > -INFINITY)) {
-          mn = mt;
-          al = mo == -INFINITY ? 0.f : __expf(mo - mn);
-          if (mo != -INFINITY) flags[0] = 1;
-        }
-        m_run[tid] = mn;
-        alpha[tid] = al;
-      }
-      __syncthreads();
-      const float vs = key_vs[j];
-      uint32_t packed[4];
-#pragma unroll
-      for (int h = 0; h < 8; h += 2) {
-        const float m0 = m_run[8 * hg + h], m1 = m_run[8 * hg + h + 1];
-        const float p0 = m0 == -INFINITY ? 0.f : __expf(sv[h] - m0);
-        const float p1 = m1 == -INFINITY ? 0.f : __expf(sv[h + 1] - m1);
-        t[h] = p0;
-        t[h + 1] = p1;
-        packed[h >> 1] = pack_f32x2(p0 * vs, p1 * vs);
-      }
-      st_shared_v4(sb + kOffP + static_cast<uint32_t>(j) * 128u + (static_cast<uint32_t>(hg ^ (j & 7)) << 4),
+      l_part = l_part * a_l + psum;
+      m_run = m_new;
+      F_run = F_new;
+      const uint32_t prow = sb + kOffP + static_cast<uint32_t>(h) * 128u;
+      const int g0 = 4 * s + kb / 8;
+      st_shared_v4(prow + (static_cast<uint32_t>(g0 ^ (h & 7)) << 4),
                    make_uint4(packed[0], packed[1], packed[2], packed[3]));
-      const float sm = warp_reduce8<false>(t, lane);
-      if ((lane & 3) == 0) red[q4 * kH + 8 * hg + (lane >> 2)] = sm;
-      __syncthreads();
-      if (tid < kH)
-        l_run[tid] = l_run[tid] * alpha[tid] + ((red[tid] + red[kH + tid]) + (red[2 * kH + tid] + red[3 * kH + tid]));
-      // rescale the output accumulated so far where the running max was raised
-      if (tile > 0 && flags[0]) {
+      st_shared_v4(prow + (static_cast<uint32_t>((g0 + 1) ^ (h & 7)) << 4),
+                   make_uint4(packed[4], packed[5], packed[6], packed[7]));
+      if (rescale) {
+        // O^T holds the output products of tiles 0 .. t-1: wait for the last of them, then scale
+        // column (head) c of every dims block of this warp's lane quarter by alpha[c]
+        const int u = t - 1;
+        got = __all_sync(0xffffffffu,
+                         wait_or_abort(bar(kBarXfree + (u & 1)), static_cast<uint32_t>(u >> 1) & 1u, abort_flag));
+        if (got) {
+          tc_fence_after();
 #pragma unroll 1
-        for (int m = 0; m < 4; ++m) {
-          const uint32_t ta = tmem + lane_base + kOCol + 64 * m + 8 * hg;
-          uint32_t o[8];
-          tmem_ld8(ta, o);
+          for (int m = 0; m < 4; ++m) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < kH; c0 += 8) {
+              const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q4) << 16) + kOCol + 64 * m + c0;
+              uint32_t o[8];
+              tmem_ld8(ta, o);
 #pragma unroll
-          for (int h = 0; h < 8; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[8 * hg + h]);
-          tmem_st8(ta, o);
+              for (int c = 0; c < 8; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha_sm[c0 + c]);
+              tmem_st8(ta, o);
+            }
+          }
         }
+        ok = bar_red<true>(1, kSoftThreads, got);
+        if (!ok) break;
       }
       fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(bar(kBarPfull + s));
     }
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) flags[0] = 0;
-
-    // ---- O^T += X^T . P^T
-    if (tid == 128) {
-      tc_fence_after();
-#pragma unroll 1
-      for (int kk = 0; kk < (n_valid + 15) / 16; ++kk) {   // consecutive MMAs go to different accumulators
-        const uint64_t bp = sdesc(sb + kOffP + kk * 2048, 8192, 1024);
+    if (!ok) {
+      *abort_flag = 1;
+    } else {
+      // the head's sum: hi row plus its lo partner (they share the maximum)
+      if (!hi_row) red_f[q4 * 32 + lane] = l_part;
+      named_sync(1, kSoftThreads);
+      if (hi_row) {
+        const float l = l_part + red_f[(q4 ^ 2) * 32 + lane];
+        reinterpret_cast<float2*>(ws.part_ml)[slot + h] = make_float2(m_run, l);
+        if (h == 0) *f_final = F_run;
+      }
+    }
+  } else {
+    // ---------------- loaders: stage tile t into stage t & 1 once the output product of tile t-2
+    //                  has released it
+    auto stage = [&](int t, Raw (&r)[2][2]) -> bool {
+      const int s = t & 1;
+      if (t >= 2 && !__all_sync(0xffffffffu, wait_or_abort(bar(kBarXfree + s),
+                                                             static_cast<uint32_t>((t >> 1) - 1) & 1u, abort_flag)))
+        return false;
+      const uint32_t xs = sb + kOffX + s * kXStage;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint64_t a = sdesc(sb + kOffX + 2 * m * kXChunk + kk * 2048, kXChunk, 1024);
-          mma_f16(tmem + kOCol + 64 * m, a, bp, kIdescPV, (tile > 0 || kk > 0) ? 1u : 0u);
+      for (int u = 0; u < 2; ++u) {
+        const int key = 2 * li + u;
+        bool win;
+        float tsc;
+        const int64_t row = row_of(t, u, &win, &tsc);
+        float v[2][8];
+        decode_granule<CT>(r[u][0], win, v[0]);
+        decode_granule<CT>(r[u][1], win, v[1]);
+        uint32_t mb = 0;
+#pragma unroll
+        for (int g = 0; g < 2; ++g)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mb = max(mb, __float_as_uint(v[g][k]) & 0x7fffffffu);
+        // a power of two that puts the key's largest magnitude in [2^8, 2^9); the key factor is
+        // its inverse times the token scale (0 marks an absent key, whose row is zeros)
+        const int sh = norm_shift(__reduce_max_sync(0xffffffffu, mb));
+        const float up = exp2i(sh);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          uint4 o;
+          o.x = pack_f32x2(v[g][0] * up, v[g][1] * up);
+          o.y = pack_f32x2(v[g][2] * up, v[g][3] * up);
+          o.z = pack_f32x2(v[g][4] * up, v[g][5] * up);
+          o.w = pack_f32x2(v[g][6] * up, v[g][7] * up);
+          st_shared_v4(xs + swz(kXChunk, key, lane + 32 * g), o);
         }
+        if (lane == 0) kf[s * kTile + key] = row >= 0 ? tsc * exp2i(-sh) : 0.f;
       }
-      mma_commit(bar);
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarXfull + s));
+      return true;
+    };
+    bool ok = true;
+    for (int t = 0; t < n_tiles && ok; t += 2) {
+      ok = stage(t, ring[0]);
+      if (ok && t + 2 < n_tiles) issue(t + 2, ring[0]);
+      if (ok && t + 1 < n_tiles) {
+        ok = stage(t + 1, ring[1]);
+        if (ok && t + 3 < n_tiles) issue(t + 3, ring[1]);
+      }
     }
-    ok = __syncthreads_and(mbar_wait(bar, phase)) != 0;
-    phase ^= 1;
-    tc_fence_after();
+    if (!ok) *abort_flag = 1;
   }
 
-  // ---- partial outputs: O^T lane = dim, column = head (warp w: lane quarter w%4, heads of
-  //      group w/4). Each head's row is stored as fp16 after division by a power of two 2^e,
-  //      e = (exponent of the row's max |o|) - 15 (at least -126), so that every value lies below
-  //      2^15 in magnitude with a relative step of 2^-11 of the row's max; e goes to part_sc.
-  if (ok) {
-    const int q4 = warp & 3, hg = warp >> 2;
-    const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
-    uint32_t o[4][8];
+  __syncthreads();  // every role done; the MMA thread has drained the tensor pipe
+  const bool aborted = *abort_flag != 0;
+  if (!aborted && warp >= kFirstLoadWarp) {
+    // ---------------- partial outputs: O^T lane = dim, column = head. Loader warp li reads its
+    //                  TMEM lane quarter and head groups li/4 and li/4 + 4. Each head's row is
+    //                  stored as fp16 after division by 2^e, e = (exponent of the row's max
+    //                  |O^T|) - 15 (at least -126): values below 2^15 with a step of 2^-11 of the
+    //                  row's max; part_sc = 2^e F.
+    tc_fence_after();
+    const int q4 = warp & 3;
+    const float F = *f_final;
+    auto load_group = [&](int hg, uint32_t (&o)[4][8]) {
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
-      tmem_ld8(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + kOCol + 64 * m + 8 * hg, o[m]);
-    float t[8];
+      for (int m = 0; m < 4; ++m)
+        tmem_ld8(tmem + (static_cast<uint32_t>(32 * q4) << 16) + kOCol + 64 * m + 8 * hg, o[m]);
+    };
+#pragma unroll 1
+    for (int gi = 0; gi < 2; ++gi) {
+      const int hg = li / 4 + 4 * gi;
+      uint32_t o[4][8];
+      load_group(hg, o);
 #pragma unroll
-    for (int h = 0; h < 8; ++h)
-      t[h] = fmaxf(fmaxf(fabsf(__uint_as_float(o[0][h])), fabsf(__uint_as_float(o[1][h]))),
-                   fmaxf(fabsf(__uint_as_float(o[2][h])), fabsf(__uint_as_float(o[3][h]))));
-    const float amax_w = warp_reduce8<true>(t, lane);
-    if ((lane & 3) == 0) red[q4 * kH + 8 * hg + (lane >> 2)] = amax_w;
-    __syncthreads();
-    if (tid < kH) {
-      const float amax = fmaxf(fmaxf(red[tid], red[kH + tid]), fmaxf(red[2 * kH + tid], red[3 * kH + tid]));
-      int ex = 0;
-      float sc = 1.f;
-      if (amax > 0.f && amax <= 3.4e38f) {   // finite, non-zero
-        frexpf(amax, &ex);                    // amax = f * 2^ex, f in [0.5, 1)
-        sc = ldexpf(1.f, ex - 15 > -126 ? ex - 15 : -126);
+      for (int c = 0; c < 8; ++c) {
+        float a = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) a = fmaxf(a, fabsf(__uint_as_float(o[m][c])));
+        a = warp_max(a);
+        if (lane == 0) epi[q4 * kH + 8 * hg + c] = a;
       }
-      alpha[tid] = sc;
-      ws.part_sc[slot + tid] = sc;
     }
-    __syncthreads();
+    named_sync(2, kLoadThreads);
+#pragma unroll 1
+    for (int gi = 0; gi < 2; ++gi) {
+      const int hg = li / 4 + 4 * gi;
+      uint32_t o[4][8];
+      load_group(hg, o);
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      const float inv = 1.f / alpha[8 * hg + h];   // exact: a power of two
-      __half* dst = reinterpret_cast<__half*>(ws.part_h) + (slot + 8 * hg + h) * kD + 32 * q4 + lane;
+      for (int c = 0; c < 8; ++c) {
+        const int hh = 8 * hg + c;
+        const float amax = fmaxf(fmaxf(epi[hh], epi[kH + hh]), fmaxf(epi[2 * kH + hh], epi[3 * kH + hh]));
+        int ex = 0;
+        float sc = 1.f;
+        if (amax > 0.f && amax <= 3.4e38f) {
+          frexpf(amax, &ex);  // amax = f * 2^ex, f in [0.5, 1)
+          sc = exp2i(ex - 15 > -126 ? ex - 15 : -126);
+        }
+        const float inv = 1.f / sc;  // exact: a power of two
+        __half* dst = reinterpret_cast<__half*>(ws.part_h) + (slot + hh) * kD + 32 * q4 + lane;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) dst[128 * m] = __float2half_rn(__uint_as_float(o[m][h]) * inv);
+        for (int m = 0; m < 4; ++m) dst[128 * m] = __float2half_rn(__uint_as_float(o[m][c]) * inv);
+        if (q4 == 0 && lane == 0) ws.part_sc[slot + hh] = sc * F;
+      }
     }
-    if (tid < kH) reinterpret_cast<float2*>(ws.part_ml)[slot + tid] = make_float2(m_run[tid], l_run[tid]);
   }
-  if (!ok) {
+  if (aborted) {
     if (tid == 0) atomicOr(status, CKV_DEV_TIMEOUT);
-    const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
     if (tid < kH) reinterpret_cast<float2*>(ws.part_ml)[slot + tid] = make_float2(-INFINITY, 0.f);
   }
-  release();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
 }
 
-template <int CT, int WT>
+template <int CT>
 cudaError_t launch_tc(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
                       const float* q, const int32_t* idx, const int32_t* cnt, int idx_stride,
                       const AttnWs& ws, uint32_t* status, cudaStream_t stream) {
-  auto kern = attn_tc_kernel<CT, WT>;
+  auto kern = attn_tc_kernel<CT>;
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(ws.splits, batch);
@@ -599,38 +803,41 @@ cudaError_t launch_tc(const LayerParams& p, int batch, const int32_t* seq_len, i
 
 }  // namespace
 
-// fp32 caches stay on the CUDA-core path: their values are neither exact in fp16 nor inside its
-// range, and fp32 arithmetic attends them as stored
+// bf16 and NVFP4 compressed caches with an FP8 window at H = 64, D = 512. fp32 caches stay on the
+// CUDA-core path: fp32 arithmetic attends them as stored.
 bool attention_tc_supported(const LayerParams& p) {
   return p.H == kH && p.D == kD && (p.comp_dtype == CKV_BF16 || p.comp_dtype == CKV_NVFP4) &&
          p.win_dtype == CKV_FP8_E4M3;
 }
 
-int attention_tc_tiles_per_split(int batch, int64_t max_keys) {
-  const int64_t tiles = static_cast<int64_t>(batch) * ((max_keys + kTile - 1) / kTile);
-  const int64_t cap = 4 * static_cast<int64_t>(sm_count());
-  int64_t t = tiles > cap ? (tiles + cap - 1) / cap : 1;
-  return static_cast<int>(t < 8 ? t : 8);
-}
-
+// Keys per split: t tiles of 32 keys, t in 1 .. 16, minimising (waves of one CTA per SM) x
+// (t + 2), the 2 standing for a split's fixed cost (query image, rows, partial write).
 int attention_tc_keys_per_split(int batch, int64_t max_keys) {
-  // half tiles (64 keys; the MMAs still run at M = 128 over the staged half) while they fit one
-  // wave: twice the CTAs, each staging half the rows
-  const int64_t halves = static_cast<int64_t>(batch) * ((max_keys + kTile / 2 - 1) / (kTile / 2));
-  if (halves <= sm_count()) return kTile / 2;
-  return kTile * attention_tc_tiles_per_split(batch, max_keys);
+  const int64_t tiles = max_keys > 0 ? (max_keys + kTile - 1) / kTile : 1;
+  const int64_t sms = sm_count();
+  int best_t = 1;
+  int64_t best = -1;
+  for (int t = 1; t <= kMaxTiles; ++t) {
+    const int64_t ctas = static_cast<int64_t>(batch) * ((tiles + t - 1) / t);
+    const int64_t cost = ((ctas + sms - 1) / sms) * (t + 2);
+    if (best < 0 || cost < best) {
+      best = cost;
+      best_t = t;
+    }
+    if (t >= tiles) break;
+  }
+  return kTile * best_t;
 }
 
 cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,
                                 int max_seq_len, const float* q, const int32_t* idx,
                                 const int32_t* cnt, int idx_stride, const AttnWs& ws,
                                 uint32_t* status, cudaStream_t stream) {
-#define CKV_TC(CT, WT) \
-  if (p.comp_dtype == CT && p.win_dtype == WT) \
-    return launch_tc<CT, WT>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);
-  CKV_TC(CKV_BF16, CKV_FP8_E4M3)
-  CKV_TC(CKV_NVFP4, CKV_FP8_E4M3)
-#undef CKV_TC
+  if (p.win_dtype != CKV_FP8_E4M3) return cudaErrorInvalidValue;
+  if (p.comp_dtype == CKV_BF16)
+    return launch_tc<CKV_BF16>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);
+  if (p.comp_dtype == CKV_NVFP4)
+    return launch_tc<CKV_NVFP4>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);
   return cudaErrorInvalidValue;
 }
 

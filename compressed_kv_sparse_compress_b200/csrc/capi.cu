@@ -300,6 +300,18 @@ int kv_compress_append(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, i
   return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
 }
 
+int kv_window_replay(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int32_t batch,
+                     const int32_t* d_seq_len, int32_t max_seq_len, const float* d_kv, const float* d_logit,
+                     uint32_t* d_status, void* stream) {
+  LayerParams p{};
+  const int st = make_params(cfg, cache, batch, max_seq_len, true, &p);
+  if (st != CKV_OK) return st;
+  if (!d_seq_len || !d_status || (p.W > 0 && (!d_kv || !d_logit || !aligned16(d_kv)))) return CKV_ERR_INVALID_ARG;
+  cudaError_t e = launch_window_replay(p, batch, d_seq_len, max_seq_len, d_kv, d_logit, d_status,
+                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+}
+
 int sparse_indexer_topk(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int32_t batch,
                         const int32_t* d_seq_len, int32_t max_seq_len, const float* d_q,
                         int32_t top_k, int32_t* d_idx, int32_t* d_cnt, float* d_scores,
@@ -387,9 +399,9 @@ int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int3
   AttnWs aw{};
   if (ws_bytes < step_ws_bytes(p, batch, max_seq_len, top_k, &iw, &aw, d_ws)) return CKV_ERR_WORKSPACE;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // append of the token at seq_len[b] - 1 side by side with the query pass (q_bar and the
-  // attention's query preparation), then selection (sparse layers) and attention
-  const QueryPrepOut prep{aw.rope, attention_tc_supported(p) ? aw.qimage : nullptr};
+  // append of the token at seq_len[b] - 1 side by side with the query pass (q_bar and the cos/sin
+  // table of the rotary pairs), then selection (sparse layers) and attention
+  const QueryPrepOut prep{aw.rope};
   // With more (request, slice) CTAs than SMs the append and the query pass run side by side in one
   // front kernel. With fewer, they stay two kernels: the front kernel's CTAs take a whole SM's
   // registers each, which keeps the next kernel's CTAs from becoming resident early (measured:
@@ -408,7 +420,8 @@ int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int3
                        prep, front);
     if (e != cudaSuccess) return CKV_ERR_CUDA;
   }
-  // the query preparation is done when the front kernel ran or the indexer's q-bar pass wrote it
+  // the cos/sin table is written when the front kernel ran or the indexer's q-bar pass wrote it
+  // (the tensor-core attention writes it itself either way)
   e = launch_attention(p, batch, d_seq_len, max_seq_len, d_q, top_k > 0 ? d_idx : nullptr,
                        top_k > 0 ? d_cnt : nullptr, top_k > 0 ? top_k : 0, d_out, aw, d_status, s,
                        front || top_k > 0);

@@ -49,6 +49,11 @@ cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_l
                           const float* logit_new, uint32_t* status, cudaStream_t stream,
                           int prev_offset = 0);
 
+// SWA bounded replay: rewrites the last min(W, L) window rows and the unfinished group's ring slots
+// of every request from kv [batch][W][D] / logit [batch][W] (row i = position L - n_w + i).
+cudaError_t launch_window_replay(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
+                                 const float* kv, const float* logit, uint32_t* status, cudaStream_t stream);
+
 // ---------------------------------------------------------------------------- indexer
 constexpr int kHistBins = 2048;  // first radix digit: the top 11 bits of the order key
 
@@ -66,18 +71,17 @@ struct IndexerWs {
 int64_t score_stride(int ratio, int max_seq_len);
 IndexerWs indexer_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len);
 
-// Outputs of the query pass that the attention of the same layer and step can take over (the
-// cos/sin table and, on the tensor-core path, the rotated fp16 query image); null: not written.
+// Output of the query pass that the attention of the same layer and step can take over: the
+// cos/sin table of the rotary pairs at the query position (null: not written).
 struct QueryPrepOut {
   double* rope;
-  uint8_t* qimage;
 };
 // skip_qbar: q_bar, the counts and the reset of the selection state are already done (by the
 // fused step's front kernel)
 cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
                            int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
                            float* scores, const IndexerWs& ws, uint32_t* status,
-                           cudaStream_t stream, QueryPrepOut prep = {nullptr, nullptr},
+                           cudaStream_t stream, QueryPrepOut prep = {nullptr},
                            bool skip_qbar = false);
 
 // Top-k of the scores a score pass wrote, with the candidate counts, the reset selection state
@@ -112,22 +116,21 @@ struct AttnWs {
   uint16_t* part_h;  // [B][S][H][D]   tensor-core path: fp16 partial outputs divided by part_sc
                      //                (same memory as part_o)
   float* part_sc;    // [B][S][H]      tensor-core path: power-of-two scale of each partial
-  bool half_parts;   // which of the two forms the splits write
-  float* part_ml;    // [B][S][H][2]   running max and sum of each split
+  bool half_parts;   // which of the two forms the splits write (the tensor-core form)
+  float* part_ml;    // [B][S][H][2]   running max and sum of each split (max in nats on the
+                     //                CUDA-core path, in base 2 on the tensor-core path)
   double* rope;      // [B][d_r/2][2]  cos, sin of each rotary pair at the query position
-  uint8_t* qimage;   // [B][H*D*2]     tensor-core path: rotated fp16 query in the swizzled
-                     //                shared-memory layout of the MMA operand
   int splits;        // S: splits per request
   int keys_per_split;
   size_t bytes;
 };
-constexpr int kQImageBytes = 64 * 512 * 2;  // H = 64, D = 512 fp16
 bool attention_tc_supported(const LayerParams& p);  // the tensor-core path serves this layer
 AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len,
                            int max_selected);
 
-// prep_done: the cos/sin table and query image are already in ws (written by the indexer's query
-// pass of the same step), so the prep kernel is not launched
+// prep_done: the cos/sin table is already in ws (written by the indexer's query pass of the same
+// step), so the CUDA-core path launches no prep kernel (the tensor-core kernel writes the table
+// itself)
 cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq_len,
                              int max_seq_len, const float* q, const int32_t* idx,
                              const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,

@@ -1,8 +1,8 @@
 // Query passes shared by the kernels of the indexer, the attention and the fused decode step's
 // front kernel: the head-averaged query q_bar of the indexer (one slice of dim pairs per call)
-// and the attention's query preparation (cos/sin table, rotated fp16 operand image). Each runs on
-// a group of 256 threads (ids tid) that synchronise through barrier bar_id (0 when the group is
-// the whole CTA).
+// and the cos/sin table of the rotary pairs at the query position (for the combine's inverse
+// rotation). Each runs on a group of 256 threads (ids tid) that synchronise through barrier
+// bar_id (0 when the group is the whole CTA).
 #pragma once
 
 #include "ckv_internal.h"
@@ -21,10 +21,8 @@ __device__ __forceinline__ void group_sync(int bar_id) {
 // [s * P, (s + 1) * P) with P = D / 2 / kQbarSlices: thread (pair k, head group g) sums its heads of
 // one pair in fp64 with all its loads in flight at once; the head groups are added in shared
 // memory, the sum rotated and scaled. The slices also reset the request's selection state.
-// With `prep` set (a fused decode step), the same pass writes what the attention's query
-// preparation would: the cos/sin table of the rotary pairs and, for H = 64 and D = 512, every
-// head's rotated query rounded to fp16 in the swizzled operand layout (chunk of 64 dims = slice,
-// row = head), with the prep kernel's arithmetic.
+// With `prep` set (a fused decode step), the same pass writes the cos/sin table of the rotary
+// pairs that the attention's query preparation would write.
 
 __device__ __forceinline__ void qbar_slice(const LayerParams& p, const int32_t* seq_len, int max_seq_len,
                                            const float* q, const IndexerWs& ws, uint32_t* status,
@@ -47,8 +45,7 @@ __device__ __forceinline__ void qbar_slice(const LayerParams& p, const int32_t* 
   const float* qb = q + static_cast<int64_t>(b) * p.H * p.D;
   const int h_lo = (p.H * g) / G, h_hi = (p.H * (g + 1)) / G;
   const bool rope_pair = pr >= first_rope && ok;
-  const bool image = prep.qimage != nullptr && ok;  // H = 64, D = 512 (checked by the caller)
-  const bool rotate = rope_pair && (g == 0 || image);
+  const bool rotate = rope_pair && g == 0;
   double s0 = 0.0, s1 = 0.0, rsn = 0.0, rcs = 1.0;
   bool have_angle = false;
   for (int h0 = h_lo; h0 < h_hi; h0 += 16) {
@@ -65,22 +62,6 @@ __device__ __forceinline__ void qbar_slice(const LayerParams& p, const int32_t* 
     for (int u = 0; u < 16; ++u) {
       s0 += v[u].x;
       s1 += v[u].y;
-    }
-    if (image) {  // head h0 + u, dims 2pr, 2pr + 1 -> chunk pr/32, row h, slot ((pr%32)/4)^(h%8), word pr%4
-      uint8_t* img = prep.qimage + static_cast<int64_t>(b) * kQImageBytes + (pr >> 5) * (64 * 128) + (pr & 3) * 4;
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int h = h0 + u;
-        if (h >= h_hi) break;
-        float x0 = v[u].x, x1 = v[u].y;
-        if (rope_pair) {
-          const double a0 = x0, a1 = x1;
-          x0 = static_cast<float>(a0 * rcs - a1 * rsn);
-          x1 = static_cast<float>(a0 * rsn + a1 * rcs);
-        }
-        const __half2 hh = __floats2half2_rn(x0, x1);
-        *reinterpret_cast<__half2*>(img + h * 128 + ((((pr & 31) >> 2) ^ (h & 7)) << 4)) = hh;
-      }
     }
   }
   if (rotate && !have_angle)  // head group 0 holds no heads when H < G
@@ -111,15 +92,10 @@ __device__ __forceinline__ void qbar_slice(const LayerParams& p, const int32_t* 
 }
 
 // Per request: cos/sin of every rotary pair at the query position L-1 (fp64 angles), for the
-// inverse rotation in the combine; on the tensor-core path also the rotated query rounded to
-// fp16, written as the 128-byte-swizzled image of the MMA operand so that each attention CTA
-// fetches it with one bulk copy.
-
-// Part `part` of request b (part 0 alone on the CUDA-core path; parts 0..7 build heads 8x .. 8x+7
-// of the tensor-core image), kPrepThreads threads with ids tid.
+// inverse rotation in the combine, by kPrepThreads threads with ids tid (part 0 of request b).
 __device__ __forceinline__ void prep_part(const LayerParams& p, const int32_t* seq_len, int max_seq_len,
-                                          const float* q, const AttnWs& ws, int part, int b, int tid,
-                                          double* rope_s, int bar_id) {
+                                          const AttnWs& ws, int part, int b, int tid) {
+  if (part != 0) return;
   const int L = seq_len[b];
   if (L < 1 || L > max_seq_len) return;
   const int n_pairs = p.d_r / 2;
@@ -127,55 +103,8 @@ __device__ __forceinline__ void prep_part(const LayerParams& p, const int32_t* s
   for (int i = tid; i < n_pairs; i += kPrepThreads) {
     double sn, cs;
     sincos(static_cast<double>(L - 1) * rope_inv_freq(p, i), &sn, &cs);
-    rope_s[2 * i] = cs;
-    rope_s[2 * i + 1] = sn;
-    if (part == 0) {
-      rope_g[2 * i] = cs;
-      rope_g[2 * i + 1] = sn;
-    }
-  }
-  if (!ws.qimage) return;
-  group_sync(bar_id);
-  // tensor-core path (H = 64, D = 512): granule g (8 dims) of head h lands at chunk g/8, row h,
-  // 16-byte slot (g % 8) ^ (h % 8) of the operand image; CTA x builds heads 8x .. 8x+7
-  constexpr int kD = 512, kGr = kD / 8, kChunk = 64 * 128;
-  const float* qb = q + static_cast<int64_t>(b) * 64 * kD;
-  uint8_t* img = ws.qimage + static_cast<int64_t>(b) * kQImageBytes;
-  const int first_rope = (kD - p.d_r) / 2;
-  for (int it0 = part * 8 * kGr; it0 < (part + 1) * 8 * kGr; it0 += 2 * kPrepThreads) {
-    float4 raw[2][2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int it = it0 + u * kPrepThreads + tid;
-      const float4* src = reinterpret_cast<const float4*>(qb + (it >> 6) * kD + 8 * (it & 63));
-      raw[u][0] = __ldg(src);
-      raw[u][1] = __ldg(src + 1);
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int it = it0 + u * kPrepThreads + tid;
-      const int h = it >> 6, g = it & 63;
-      float v[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
-                    raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int pr = 4 * g + k;
-        if (pr >= first_rope) {
-          const double cs = rope_s[2 * (pr - first_rope)], sn = rope_s[2 * (pr - first_rope) + 1];
-          const double x0 = v[2 * k], x1 = v[2 * k + 1];
-          v[2 * k] = static_cast<float>(x0 * cs - x1 * sn);
-          v[2 * k + 1] = static_cast<float>(x0 * sn + x1 * cs);
-        }
-      }
-      uint32_t w[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        __half2 hh = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
-        w[k] = *reinterpret_cast<uint32_t*>(&hh);
-      }
-      const uint32_t off = static_cast<uint32_t>(g >> 3) * kChunk + h * 128 + (((g & 7) ^ (h & 7)) << 4);
-      *reinterpret_cast<uint4*>(img + off) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
+    rope_g[2 * i] = cs;
+    rope_g[2 * i + 1] = sn;
   }
 }
 

@@ -51,6 +51,12 @@ class DecodeLayer:
                              cu_new=cu_new, max_new=max_new, max_seq_len=self.max_seq_len,
                              stream=stream)
 
+    def replay_window(self, seq_len, kv, logit, stream=None):
+        """SWA bounded replay: the recomputed raw tokens of the last min(W, L) positions of each
+        request (kv [batch][W][D], logit [batch][W]) rewrite its window and unfinished group."""
+        B.kv_window_replay(self.cfg, self.cache, seq_len, kv, logit, self.status,
+                           max_seq_len=self.max_seq_len, stream=stream)
+
     def select(self, seq_len, q, scores=None, stream=None):
         B.sparse_indexer_topk(self.cfg, self.cache, seq_len, self.max_seq_len, q, self.top_k,
                               self.idx, self.cnt, self.ws_index, self.status, scores=scores,

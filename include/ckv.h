@@ -179,6 +179,27 @@ int kv_compress_append(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, i
                        uint32_t* d_status, void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* SWA bounded replay ([CZ] section "Proc je obnova sliding-window cache draha": after a
+ * prefix-cache hit only the last window is run through the model again, and the dependence on
+ * positions before it is cut; [CZ] section "Polovina vrstev nemusi cist cely prompt" names the
+ * switch). The model recomputes the window's K=V vectors; this call puts them in the cache.
+ *
+ * For request b with L = seq_len[b] and n_w = min(W, L): the raw (un-rotated) tokens of positions
+ * L - n_w .. L - 1 are rotated at their own positions and written to the window cache with the
+ * rules of kv_compress_append; those in the unfinished group [floor(L/r) r, L) also go to the
+ * residue ring (slot = position % r) with their compressor logits, so that the next append folds
+ * them. Compressed entries are not touched (they come from the prefix cache). Ring slots of the
+ * unfinished group's positions before L - n_w (only possible when r - 1 > W) are left as they are.
+ *
+ *   d_seq_len   [batch] int32, 1 <= L <= max_seq_len (else CKV_DEV_BAD_LENGTH, request skipped).
+ *   d_kv        [batch][W][D] fp32: row i of request b is position L - n_w + i (rows >= n_w unused).
+ *   d_logit     [batch][W] fp32 compressor logits, same rows.
+ * The window table must map the blocks of positions [L - n_w, L). W == 0 enqueues nothing. */
+int kv_window_replay(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int32_t batch,
+                     const int32_t* d_seq_len, int32_t max_seq_len, const float* d_kv, const float* d_logit,
+                     uint32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
 /* Step 2: the sparse MQA indexer and top-k ([HR] section A: sparse attention over the top-k
  * compressed tokens; [CZ] section C: "Sparse MQA logits" scores the candidate positions).
  *
@@ -253,9 +274,9 @@ int sparse_indexer_topk_noalloc(const ckv_layer_cfg* cfg, const ckv_layer_cache*
  * shared K=V attention); [CZ] section C credits the speed-up to fused kernels. One token per
  * request is appended at position seq_len[b] - 1, the layer's top_k entries are selected
  * (top_k > 0, CSA) or all entries are attended (top_k == 0, HCA), and the output is written.
- * Compared with the three calls, the query pass of the indexer also writes the attention's query
- * preparation (cos/sin table, rotated fp16 query image), so one kernel launch is saved on sparse
- * layers; every result is bit-identical to the three calls'.
+ * Compared with the three calls, the append of the new token runs beside the indexer's query pass
+ * (in one kernel when the batch fills the GPU), and that pass also writes the cos/sin table the
+ * attention's merge needs; every result is bit-identical to the three calls'.
  *
  *   d_seq_len    [batch] int32: L_b including the new token (1 .. max_seq_len).
  *   d_q          [batch][H][D] fp32 raw query; d_kv_new [batch][D] fp32 raw token; d_logit_new

@@ -1,10 +1,10 @@
 """ckv_decode_step: append, select and attend of one layer in one call.
 
-The fused call runs the same kernels as the three calls except that the indexer's query pass also
-writes the attention's query preparation (cos/sin table and, for H = 64 and D = 512, the rotated
-fp16 query image) with the prep kernel's arithmetic, so every result must be bit-identical to the
-three calls': the output, the selection and every byte the append writes. Each side works on its
-own copy of the same generated pools.
+The fused call runs the same kernels as the three calls except that the append runs beside the
+indexer's query pass (one front kernel on large batches) and that pass also writes the cos/sin
+table of the rotary pairs with the prep kernel's arithmetic, so every result must be bit-identical
+to the three calls': the output, the selection and every byte the append writes. Each side works
+on its own copy of the same generated pools.
 """
 
 import numpy as np
