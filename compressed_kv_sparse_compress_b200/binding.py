@@ -39,7 +39,7 @@ EXPORTS = (
     "sparse_indexer_topk", "compressed_window_attention", "ckv_status_str", "ckv_launch_count",
     "ckv_profile_events", "sparse_indexer_topk_noalloc", "ckv_decode_step_workspace_bytes",
     "ckv_decode_step", "kv_index_append", "ckv_mh_indexer_workspace_bytes", "sparse_mh_indexer_topk",
-    "kv_window_replay",
+    "kv_window_replay", "ckv_debug_force_timeout",
 )
 CKV_PROF_SCORE, CKV_PROF_ATTENTION = 0, 1
 
@@ -131,6 +131,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ckv_status_str.restype = ctypes.c_char_p
     lib.ckv_profile_events.argtypes = [ctypes.c_int, vp, vp]
     lib.ckv_profile_events.restype = ctypes.c_int
+    lib.ckv_debug_force_timeout.argtypes = [i32]
+    lib.ckv_debug_force_timeout.restype = ctypes.c_int
     lib.ckv_launch_count.argtypes = []
     lib.ckv_launch_count.restype = ctypes.c_uint64
     for name in ("kv_block_pool_create", "kv_block_pool_destroy", "kv_block_alloc",
@@ -147,6 +149,11 @@ def status_str(status: int) -> str:
 
 def launch_count() -> int:
     return int(load_library().ckv_launch_count())
+
+
+def debug_force_timeout(request: int) -> None:
+    """Test hook of the device failure path (ckv_debug_force_timeout); -1 turns it off."""
+    _check("ckv_debug_force_timeout", load_library().ckv_debug_force_timeout(request))
 
 
 def profile_events(which: int, begin=None, end=None) -> None:

@@ -47,6 +47,11 @@
 #include "ckv_ptx.cuh"
 
 namespace ckv {
+
+// Failure-path hook for tests (ckv_debug_force_timeout): the request whose MMA issuers wait on a
+// barrier that nothing completes, -1 for none.
+__device__ int g_attn_forced_timeout = -1;
+
 namespace {
 
 constexpr int kH = 64;
@@ -208,8 +213,9 @@ __device__ __forceinline__ bool bar_red(int id, int n, bool v) {
 
 // bounded wait for the completion of the barrier phase with parity `phase`; also gives up once
 // another role has raised the abort flag
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t phase, volatile int* abort_flag) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t phase, volatile int* abort_flag,
+                                              uint32_t limit = kWaitLimit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, phase)) return true;
     if ((i & 255u) == 255u && *abort_flag) return false;
   }
@@ -517,7 +523,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         mma_commit(bar(kBarXfree + s));
         return true;
       };
-      bool ok = true;
+      // the failure-path hook: a wait on the drain barrier, which nothing completes before the
+      // first MMA, runs out and the CTA takes its failure path
+      bool ok = g_attn_forced_timeout != b || wait_or_abort(bar(kBarDrain), 0, abort_flag, 1u << 12);
       for (int t = 0; t < n_tiles && ok; ++t) {
         const int s = t & 1;
         ok = wait_or_abort(bar(kBarXfull + s), static_cast<uint32_t>(t >> 1) & 1u, abort_flag) &&
@@ -827,6 +835,10 @@ int attention_tc_keys_per_split(int batch, int64_t max_keys) {
     if (t >= tiles) break;
   }
   return kTile * best_t;
+}
+
+cudaError_t attention_force_timeout(int request) {
+  return cudaMemcpyToSymbol(g_attn_forced_timeout, &request, sizeof(int));
 }
 
 cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,

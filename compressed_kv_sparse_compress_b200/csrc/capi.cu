@@ -498,6 +498,11 @@ const char* ckv_status_str(int status) {
 
 uint64_t ckv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+int ckv_debug_force_timeout(int32_t request) {
+  if (request < -1) return CKV_ERR_INVALID_ARG;
+  return attention_force_timeout(request) == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
+}
+
 int ckv_profile_events(int which, void* ev_begin, void* ev_end) {
   if (which != CKV_PROF_SCORE && which != CKV_PROF_ATTENTION) return CKV_ERR_INVALID_ARG;
   if ((ev_begin == nullptr) != (ev_end == nullptr)) return CKV_ERR_INVALID_ARG;

@@ -125,6 +125,8 @@ struct AttnWs {
   size_t bytes;
 };
 bool attention_tc_supported(const LayerParams& p);  // the tensor-core path serves this layer
+// Failure-path hook of the tensor-core attention (request index, -1: off); see ckv_debug_force_timeout.
+cudaError_t attention_force_timeout(int request);
 AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len,
                            int max_selected);
 

@@ -366,6 +366,15 @@ const char* ckv_status_str(int status);
 /* Number of kernel launches enqueued by this process since load (all entry points). */
 uint64_t ckv_launch_count(void);
 
+/* Failure-path hook for tests. While request >= 0, the lane that issues the tensor-core MMAs of
+ * every attention CTA of that request (tensor-core layers: H = 64, D = 512, bf16 or NVFP4
+ * compressed cache, FP8 window) first waits on a barrier that nothing completes; the bounded wait
+ * runs out, the CTA takes its failure path (nothing is issued, CKV_DEV_TIMEOUT is set, its
+ * partial is marked empty) and that request's output is zero, while the other requests and the
+ * CUDA context are unaffected. request = -1 turns it off (the default). The setting is a device
+ * variable of the current device, written with a blocking copy; not thread-safe. */
+int ckv_debug_force_timeout(int32_t request);
+
 /* Diagnostic timing. While set, every later call records the CUDA events ev_begin (just before)
  * and ev_end (just after) the launch of one kernel, on the call's stream:
  *   CKV_PROF_SCORE      the scoring kernel of sparse_indexer_topk
