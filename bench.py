@@ -388,6 +388,9 @@ def measure(ckv, args, w: S.Workload, dev, ws: int, rank: int, cpu_leg: bool) ->
                   for li in range(len(w.layers)) if takes(w.layers[li])] for _ in range(args.steps)]
         kst = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
+        for pair in kst + [x for row in pairs for x in row]:  # CUDA events are created on first record
+            for e in pair:
+                e.record(stream)
         barrier()
         for i in range(args.steps):
             flush_l2()
@@ -469,6 +472,9 @@ def measure(ckv, args, w: S.Workload, dev, ws: int, rank: int, cpu_leg: bool) ->
             torch.cuda.synchronize()
     eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    for pair in eev:
+        for e in pair:
+            e.record(stream)
     barrier()
     for i in range(args.steps):
         flush_l2()
