@@ -358,7 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   auto bar = [&](int i) { return sb + kOffBar + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffTmem);
 
-  const int b = blockIdx.y, split = blockIdx.x;
+  // requests on x so that the first split of every request is launched first and the splits that
+  // find no keys (short requests of a mixed batch) come last
+  const int b = blockIdx.x, split = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ---- set-up that reads no global memory, before waiting for the previous kernel
@@ -375,11 +377,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     *f_final = 0.f;
     fence_proxy_async();
   }
-  if (warp == kMmaWarp) tmem_alloc(sb + kOffTmem, kTmemCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
   griddep_wait();
   griddep_launch();
 
@@ -399,15 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     rope_g[2 * tid + 1] = sn;
   }
   const int64_t k_begin = static_cast<int64_t>(split) * ws.keys_per_split;
-  if (k_begin >= kl.n_keys) {  // nothing to attend (uniform across the CTA)
-    tc_fence_before();
-    __syncthreads();
-    if (warp == kMmaWarp) {
-      tc_fence_after();
-      tmem_dealloc(tmem, kTmemCols);
-    }
-    return;
-  }
+  if (k_begin >= kl.n_keys) return;  // nothing to attend (uniform across the CTA; nothing held)
+  if (warp == kMmaWarp) tmem_alloc(sb + kOffTmem, kTmemCols);
+  tc_fence_before();
+  __syncthreads();  // barrier initialisation and the tensor memory address
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
   const int nk = static_cast<int>(min(kl.n_keys - k_begin, static_cast<int64_t>(ws.keys_per_split)));
   const int n_tiles = (nk + kTile - 1) / kTile;
   const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
@@ -804,7 +798,7 @@ cudaError_t launch_tc(const LayerParams& p, int batch, const int32_t* seq_len, i
   auto kern = attn_tc_kernel<CT>;
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(ws.splits, batch);
+  dim3 grid(batch, ws.splits);
   return launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, stream, p, seq_len, max_seq_len, q, idx,
                        cnt, idx_stride, ws, status);
 }
