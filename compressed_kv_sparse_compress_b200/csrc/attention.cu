@@ -25,7 +25,7 @@ int attention_tc_keys_per_split(int batch, int64_t max_keys);
 cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,
                                 int max_seq_len, const float* q, const int32_t* idx,
                                 const int32_t* cnt, int idx_stride, const AttnWs& ws,
-                                uint32_t* status, cudaStream_t stream);
+                                uint32_t* status, cudaStream_t stream, bool rope_ready);
 
 namespace {
 
@@ -466,7 +466,7 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
   }
   prof_begin(kProfAttention, stream);
   if (attention_tc_supported(p)) {
-    e = launch_attention_tc(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);
+    e = launch_attention_tc(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream, prep_done);
   } else {
     switch (p.D) {
       case 64: e = launch_simt_d<64>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream); break;

@@ -94,7 +94,8 @@ constexpr uint32_t kOffRed = kOffKf + 2 * kTile * 4;     // float[2][4][32]: max
 constexpr uint32_t kOffAlpha = kOffRed + 2 * 4 * 32 * 4; // float[64]: O^T rescale per head
 constexpr uint32_t kOffQs = kOffAlpha + kH * 4;          // float[64]: query scale g_h per head
 constexpr uint32_t kOffEpi = kOffQs + kH * 4;            // float[4][64]: output amax per lane quarter
-constexpr uint32_t kOffMisc = kOffEpi + 4 * kH * 4;      // int abort; float F
+constexpr uint32_t kOffRope = kOffEpi + 4 * kH * 4;      // double[256][2]: cos, sin per rotary pair
+constexpr uint32_t kOffMisc = kOffRope + 256 * 16;       // int abort; float F
 constexpr uint32_t kOffBar = kOffMisc + 16;              // 11 mbarriers
 constexpr uint32_t kOffTmem = kOffBar + 11 * 8;
 constexpr uint32_t kSmemUsed = kOffTmem + 8;
@@ -341,10 +342,11 @@ __device__ __forceinline__ int64_t key_row(const LayerParams& p, const Keys& kl,
 
 // ------------------------------------------------------------------------------------ kernel
 
+// rope_ready: the step's query pass already wrote the cos/sin table into ws.rope
 template <int CT>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const float* q, const int32_t* idx,
-    const int32_t* cnt, int idx_stride, AttnWs ws, uint32_t* status) {
+    const int32_t* cnt, int idx_stride, AttnWs ws, uint32_t* status, bool rope_ready) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(base);
@@ -387,14 +389,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   kl.n_sel = !live ? 0 : idx ? min(static_cast<int64_t>(max(cnt[b], 0)), static_cast<int64_t>(idx_stride)) : kl.n_c;
   kl.n_win = live ? min(p.W, kl.L) : 0;
   kl.n_keys = kl.n_win + kl.n_sel;
-  // the cos/sin of every rotary pair at the query position, for the combine's inverse rotation
-  if (live && split == 0 && tid < p.d_r / 2) {
-    double sn, cs;
-    sincos(static_cast<double>(kl.L - 1) * rope_inv_freq(p, tid), &sn, &cs);
-    double* rope_g = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
-    rope_g[2 * tid] = cs;
-    rope_g[2 * tid + 1] = sn;
-  }
   const int64_t k_begin = static_cast<int64_t>(split) * ws.keys_per_split;
   if (k_begin >= kl.n_keys) return;  // nothing to attend (uniform across the CTA; nothing held)
   if (warp == kMmaWarp) tmem_alloc(sb + kOffTmem, kTmemCols);
@@ -402,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   __syncthreads();  // barrier initialisation and the tensor memory address
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  double* rope_sm = reinterpret_cast<double*>(base + kOffRope);
   const int nk = static_cast<int>(min(kl.n_keys - k_begin, static_cast<int64_t>(ws.keys_per_split)));
   const int n_tiles = (nk + kTile - 1) / kTile;
   const int64_t slot = (static_cast<int64_t>(b) * ws.splits + split) * kH;
@@ -430,6 +425,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       r[u][1] = load_granule<CT>(p, row, win, lane + 32);
     }
   };
+  if (warp < kSoftWarps) {
+    // the cos/sin of every rotary pair at the query position L-1 (fp64 angles), one pair per
+    // thread: taken from the step's table when its query pass wrote it, else computed here (and
+    // stored by split 0 for the combine's inverse rotation)
+    double* rope_g = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
+    for (int i = tid; i < p.d_r / 2; i += kSoftThreads) {
+      double sn, cs;
+      if (rope_ready) {
+        cs = rope_g[2 * i];
+        sn = rope_g[2 * i + 1];
+      } else {
+        sincos(static_cast<double>(kl.L - 1) * rope_inv_freq(p, i), &sn, &cs);
+        if (split == 0) {
+          rope_g[2 * i] = cs;
+          rope_g[2 * i + 1] = sn;
+        }
+      }
+      rope_sm[2 * i] = cs;
+      rope_sm[2 * i + 1] = sn;
+    }
+  }
   if (warp >= kFirstLoadWarp) {
     const int t = lane >> 1, u = lane & 1;
     const int kloc = t * kTile + 2 * li + u;
@@ -441,7 +457,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     }
     issue(0, ring[0]);
     if (n_tiles > 1) issue(1, ring[1]);
-
+  }
+  __syncthreads();  // the rotary table
+  if (warp >= kFirstLoadWarp) {
     // query image, heads 4 li .. 4 li + 3: lane l holds dims 16 l .. 16 l + 15 (granules 2l,
     // 2l + 1 of chunk l/4); the rotary pairs 8 l .. 8 l + 7 are rotated at the query position L-1
     // (fp64 angles); hi rows are h, lo rows 64 + h
@@ -460,12 +478,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         x[4 * k + 3] = v.w;
       }
       if (8 * lane + 7 >= first_rope) {
-#pragma unroll 1
+#pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int pr = 8 * lane + k;
           if (pr >= first_rope) {
-            double rs, rc;
-            sincos(static_cast<double>(kl.L - 1) * rope_inv_freq(p, pr - first_rope), &rs, &rc);
+            const double rc = rope_sm[2 * (pr - first_rope)], rs = rope_sm[2 * (pr - first_rope) + 1];
             const double a0 = x[2 * k], a1 = x[2 * k + 1];
             x[2 * k] = static_cast<float>(a0 * rc - a1 * rs);
             x[2 * k + 1] = static_cast<float>(a0 * rs + a1 * rc);
@@ -794,13 +811,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
 template <int CT>
 cudaError_t launch_tc(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
                       const float* q, const int32_t* idx, const int32_t* cnt, int idx_stride,
-                      const AttnWs& ws, uint32_t* status, cudaStream_t stream) {
+                      const AttnWs& ws, uint32_t* status, cudaStream_t stream, bool rope_ready) {
   auto kern = attn_tc_kernel<CT>;
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(batch, ws.splits);
   return launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, stream, p, seq_len, max_seq_len, q, idx,
-                       cnt, idx_stride, ws, status);
+                       cnt, idx_stride, ws, status, rope_ready);
 }
 
 }  // namespace
@@ -838,12 +855,14 @@ cudaError_t attention_force_timeout(int request) {
 cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,
                                 int max_seq_len, const float* q, const int32_t* idx,
                                 const int32_t* cnt, int idx_stride, const AttnWs& ws,
-                                uint32_t* status, cudaStream_t stream) {
+                                uint32_t* status, cudaStream_t stream, bool rope_ready) {
   if (p.win_dtype != CKV_FP8_E4M3) return cudaErrorInvalidValue;
   if (p.comp_dtype == CKV_BF16)
-    return launch_tc<CKV_BF16>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);
+    return launch_tc<CKV_BF16>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream,
+                               rope_ready);
   if (p.comp_dtype == CKV_NVFP4)
-    return launch_tc<CKV_NVFP4>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream);
+    return launch_tc<CKV_NVFP4>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream,
+                                rope_ready);
   return cudaErrorInvalidValue;
 }
 
