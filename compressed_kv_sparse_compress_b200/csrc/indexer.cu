@@ -499,14 +499,17 @@ __device__ DigitSel candidate_digit_pass(const uint2* cand, uint32_t m, uint32_t
   return DigitSel{out[0], out[1]};
 }
 
+// boundary-bin candidates that the finish kernel keeps in shared memory for its digit passes (the
+// first digit's boundary bin holds about 1.5% of a request's candidates at 262144 of them)
+constexpr uint32_t kFinishCandSmem = 16384;
+
 __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, IndexerWs ws,
                                                                      int64_t stride, int32_t* idx,
                                                                      int32_t* cnt) {
   griddep_wait();
   griddep_launch();
-  constexpr uint32_t kCandSmem = 2048;  // boundary-bin candidates kept in shared memory
   __shared__ uint32_t h[kHistBins];
-  __shared__ uint2 cand_s[kCandSmem];
+  extern __shared__ uint2 cand_s[];  // up to kFinishCandSmem boundary-bin candidates
   __shared__ uint32_t sh[32];
   __shared__ uint2 bnd;
   const int b = blockIdx.x;
@@ -522,7 +525,7 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, 
     uint32_t need = static_cast<uint32_t>(k_eff) - r1.y;
     const uint32_t m = ws.cand_cnt[b];
     const uint2* cand = ws.cand + static_cast<int64_t>(b) * stride;
-    if (m <= kCandSmem) {
+    if (m <= kFinishCandSmem) {
       for (uint32_t i = threadIdx.x; i < m; i += blockDim.x) cand_s[i] = __ldcg(cand + i);
       __syncthreads();
       cand = cand_s;
@@ -802,7 +805,10 @@ cudaError_t launch_topk(const LayerParams& p, int batch, int max_seq_len, int to
   dim3 mgrid(static_cast<unsigned>(nmax > 0 ? (nmax + kMarkChunk - 1) / kMarkChunk : 1), batch);
   cudaError_t e = launch_kernel(topk_mark_kernel, mgrid, dim3(kThreads), 0, stream, sc, stride, top_k, ws);
   if (e != cudaSuccess) return e;
-  return launch_kernel(topk_finish_kernel, dim3(batch), dim3(kFinishThreads), 0, stream, top_k, ws, stride,
+  const int smem = static_cast<int>(kFinishCandSmem * sizeof(uint2));
+  e = allow_smem(reinterpret_cast<const void*>(topk_finish_kernel), smem);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(topk_finish_kernel, dim3(batch), dim3(kFinishThreads), smem, stream, top_k, ws, stride,
                        idx, cnt);
 }
 
