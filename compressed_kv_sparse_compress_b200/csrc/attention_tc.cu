@@ -212,13 +212,13 @@ __device__ __forceinline__ bool bar_red(int id, int n, bool v) {
   return out != 0;
 }
 
-// bounded wait for the completion of the barrier phase with parity `phase`; also gives up once
-// another role has raised the abort flag
+// bounded wait for the completion of the barrier phase with parity `phase` (polls that suspend the
+// thread, ckv_ptx.cuh); also gives up once another role has raised the abort flag
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t phase, volatile int* abort_flag,
                                               uint32_t limit = kWaitLimit) {
   for (uint32_t i = 0; i < limit; ++i) {
-    if (mbar_try_wait(bar, phase)) return true;
-    if ((i & 255u) == 255u && *abort_flag) return false;
+    if (mbar_try_wait_sleep(bar, phase, kWaitSuspendNs)) return true;
+    if (*abort_flag) return false;
   }
   return false;
 }
@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       };
       // the failure-path hook: a wait on the drain barrier, which nothing completes before the
       // first MMA, runs out and the CTA takes its failure path
-      bool ok = g_attn_forced_timeout != b || wait_or_abort(bar(kBarDrain), 0, abort_flag, 1u << 12);
+      bool ok = g_attn_forced_timeout != b || wait_or_abort(bar(kBarDrain), 0, abort_flag, 16);
       for (int t = 0; t < n_tiles && ok; ++t) {
         const int s = t & 1;
         ok = wait_or_abort(bar(kBarXfull + s), static_cast<uint32_t>(t >> 1) & 1u, abort_flag) &&

@@ -5,7 +5,11 @@
 
 namespace ckv {
 
-constexpr uint32_t kWaitLimit = 1u << 22;  // polls before a bounded wait gives up
+// A bounded wait polls an mbarrier with try_wait and a suspend-time hint: a poll returns as soon as
+// the phase completes, else after at most kWaitSuspendNs with the thread suspended (it takes no
+// issue slots meanwhile); after kWaitLimit polls (a few seconds) the wait gives up.
+constexpr uint32_t kWaitLimit = 1u << 15;
+constexpr uint32_t kWaitSuspendNs = 100000;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -34,10 +38,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
   return ok != 0;
 }
 
+// one poll that may suspend the thread for up to `ns` nanoseconds while the phase is incomplete
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t phase, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(phase), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // bounded wait for the completion of the barrier phase with parity `phase`
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
   for (uint32_t i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, phase)) return true;
+    if (mbar_try_wait_sleep(bar, phase, kWaitSuspendNs)) return true;
   return false;
 }
 

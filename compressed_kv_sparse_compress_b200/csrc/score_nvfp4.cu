@@ -141,11 +141,12 @@ __device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
 
 __device__ __forceinline__ uint32_t half2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
-// bounded wait that also gives up once another role has raised the abort flag
+// bounded wait (polls that suspend the thread, ckv_ptx.cuh) that also gives up once another role
+// has raised the abort flag
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t phase, volatile int* abort_flag) {
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (mbar_try_wait(bar, phase)) return true;
-    if ((i & 255u) == 255u && *abort_flag) return false;
+    if (mbar_try_wait_sleep(bar, phase, kWaitSuspendNs)) return true;
+    if (*abort_flag) return false;
   }
   return false;
 }
