@@ -545,15 +545,21 @@ __global__ void __launch_bounds__(2 * kAppendThreads, 1) step_front_kernel(
   griddep_launch();
   __shared__ AppendDecodeSmem sm;
   __shared__ double qsm[512];  // q_bar partial sums [256][2]
+  __shared__ double rope_tmp[2 * kQiMaxRopePairs];
   const int x = blockIdx.x, b = blockIdx.y;
   if (threadIdx.x < kAppendThreads) {
     if (x < app_slices) append_decode_slice(a, x, b, threadIdx.x, 1, sm);
   } else if (kSparse) {
-    if (x < kQbarSlices)
+    if (x < kQbarSlices) {
       qbar_slice(a.p, a.prev_len, a.max_seq_len, q, iws, a.status, prep, x, b, threadIdx.x - kAppendThreads,
                  reinterpret_cast<double(*)[2]>(qsm), 2);
+      if (prep.qimage)  // the attention's query image, heads 8 x .. 8 x + 7
+        qimage_part(a.p, a.prev_len, a.max_seq_len, q, prep, x, b, threadIdx.x - kAppendThreads, rope_tmp, 2);
+    }
   } else if (x < prep_parts) {
     prep_part(a.p, a.prev_len, a.max_seq_len, aws, x, b, threadIdx.x - kAppendThreads);
+    if (prep.qimage)
+      qimage_part(a.p, a.prev_len, a.max_seq_len, q, prep, x, b, threadIdx.x - kAppendThreads, rope_tmp, 2);
   }
 }
 
@@ -566,7 +572,7 @@ cudaError_t launch_step_front(const LayerParams& p, int batch, const int32_t* se
   // the new token of request b is at position seq_len[b] - 1
   const AppendArgs a{p, seq_len, nullptr, max_seq_len, kv_new, logit_new, status, -1};
   const int app_slices = p.D / 2 < kSlicePairs ? 1 : p.D / 2 / kSlicePairs;
-  const int prep_parts = 1;
+  const int prep_parts = prep.qimage ? kQiHeads / 8 : 1;  // the rotary table; the query image by 8 heads
   const int other = sparse ? kQbarSlices : prep_parts;
   const dim3 grid(app_slices > other ? app_slices : other, batch);
   if (sparse)

@@ -17,6 +17,7 @@
 
 #include "ckv_internal.h"
 #include "query_prep.cuh"
+#include "qimage.cuh"
 #include "ckv_ptx.cuh"
 
 namespace ckv {
@@ -25,7 +26,7 @@ int attention_tc_keys_per_split(int batch, int64_t max_keys);
 cudaError_t launch_attention_tc(const LayerParams& p, int batch, const int32_t* seq_len,
                                 int max_seq_len, const float* q, const int32_t* idx,
                                 const int32_t* cnt, int idx_stride, const AttnWs& ws,
-                                uint32_t* status, cudaStream_t stream, bool rope_ready);
+                                uint32_t* status, cudaStream_t stream, bool early, bool rope_ready);
 
 namespace {
 
@@ -284,132 +285,107 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u) {
   return __half22float2(__half2(hr));
 }
 
-// Merge for the tensor-core path (H = 64, D = 512, fp16 partials O_s / c_s, maxima in base 2): one CTA per
-// (request, group of kGH heads). Each split's partial rows of the group are 4 KB of contiguous
-// memory; up to kGS splits per round are bulk-copied into shared memory while the block reduces
-// their (m, l) per head, and thread t then merges dims 8 (t % 64) .. 8 (t % 64) + 7 of head
-// t / 64 of the group from shared memory (running max and sums rescaled between rounds). The
-// shared memory holds the rounds' rows: min(splits, kGS) x 4 KB.
-constexpr int kGH = 4;
-constexpr int kGS = 48;  // splits per round (48 x 4 KB = 192 KB of shared memory)
+// Merge for the tensor-core path (H = 64, D = 512): split s of request b holds O_s as fp16 rows of 64
+// heads per dim (part_h[b][s][d][h], head h divided by part_sc[b][s][h]) and (m, l) per head with
+// the maximum in base 2. One CTA per (request, block of 32 dims); thread t merges heads 2 (t % 32),
+// 2 (t % 32) + 1 over dims 4 (t / 32) .. 4 (t / 32) + 3 of the block, so that a warp reads 128
+// contiguous bytes per dim. Each thread keeps its own running maximum, sum and accumulators (no
+// barrier), reading the splits' partials and weights from L2 a few splits at a time.
 constexpr int kGThreads = 256;
 constexpr int kGDim = 512;
-constexpr uint32_t kGRow = kGH * kGDim * 2;
+constexpr int kGHeads = 64;
+constexpr int kGDimsPerCta = 32;
+constexpr int kGBatch = 4;  // splits whose loads are in flight together
 
-__global__ void __launch_bounds__(kGThreads, 1) attn_combine_tc_kernel(
+__global__ void __launch_bounds__(kGThreads) attn_combine_tc_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const int32_t* cnt, bool sparse,
-    int idx_stride, int gs, AttnWs ws, float* out, uint32_t* status) {
+    int idx_stride, AttnWs ws, float* out, uint32_t* status) {
   griddep_wait();
   griddep_launch();
-  extern __shared__ __align__(128) uint8_t cs_raw[];  // [gs][kGH][kGDim] fp16
-  __shared__ float wts[kGS][kGH];
-  __shared__ float red[2][kGThreads / 32];
-  __shared__ __align__(8) uint64_t bar_storage;
-  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int hh = tid >> 6, t64 = tid & 63;
-  const int h = g * kGH + hh;
-  float4* o = reinterpret_cast<float4*>(out + (static_cast<int64_t>(b) * p.H + h) * kGDim + 8 * t64);
+  const int blk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int hp = tid & 31, d0 = kGDimsPerCta * blk + 4 * (tid >> 5);
+  float4* o0 = reinterpret_cast<float4*>(out + (static_cast<int64_t>(b) * kGHeads + 2 * hp) * kGDim + d0);
+  float4* o1 = o0 + kGDim / 4;
   const int L = seq_len[b];
   if (L < 1 || L > max_seq_len) {
-    if (g == 0 && tid == 0) atomicOr(status, CKV_DEV_BAD_LENGTH);
-    o[0] = o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (blk == 0 && tid == 0) atomicOr(status, CKV_DEV_BAD_LENGTH);
+    *o0 = *o1 = make_float4(0.f, 0.f, 0.f, 0.f);
     return;
   }
-  const uint32_t bar = smem_u32(&bar_storage);
-  if (tid == 0) mbar_init(bar, 1);
-  __syncthreads();
   const KeyList kl = key_list(p, L, cnt, sparse, idx_stride, b);
   const int ns = static_cast<int>((kl.n_keys + ws.keys_per_split - 1) / ws.keys_per_split);
   const int64_t base = static_cast<int64_t>(b) * ws.splits;
-  const uint8_t* src = reinterpret_cast<const uint8_t*>(ws.part_h + (base * p.H + g * kGH) * kGDim);
-  const int64_t split_bytes = static_cast<int64_t>(p.H) * kGDim * 2;
-  const float2* ml = reinterpret_cast<const float2*>(ws.part_ml);
-  float M = -INFINITY, Z = 0.f, acc[8];
+  const float4* ml = reinterpret_cast<const float4*>(ws.part_ml);           // (m, l) of 2 heads
+  const float2* scp = reinterpret_cast<const float2*>(ws.part_sc);          // scales of 2 heads
+  const uint32_t* ph = reinterpret_cast<const uint32_t*>(ws.part_h);        // fp16 pairs of heads
+  float M[2] = {-INFINITY, -INFINITY}, Z[2] = {0.f, 0.f}, acc[2][4];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
-  uint32_t phase = 0;
-  bool ok = true;
-  for (int s0 = 0; s0 < ns && ok; s0 += gs) {
-    const int nb = min(gs, ns - s0);
-    if (tid == 0) {
-      fence_proxy_async();  // earlier rounds' reads of the buffer come before the copies
-      mbar_expect_tx(bar, static_cast<uint32_t>(nb) * kGRow);
-      for (int u = 0; u < nb; ++u)
-        bulk_g2s(smem_u32(cs_raw + u * kGRow), src + (s0 + u) * split_bytes, kGRow, bar);
-    }
-    // weights of this round's splits, per head (64 threads per head: 2 warps)
-    float2 v = make_float2(-INFINITY, 0.f);
-    float scv = 0.f;
-    if (t64 < nb) {
-      v = __ldcg(ml + (base + s0 + t64) * p.H + h);
-      scv = __ldcg(ws.part_sc + (base + s0 + t64) * p.H + h);
-    }
-    const bool live = t64 < nb && v.y > 0.f;  // l = 0: the split holds no keys (or gave up)
-    const float mw = warp_max(live ? v.x : -INFINITY);
-    if (lane == 0) red[0][warp] = mw;
-    __syncthreads();
-    const float Mn = fmaxf(M, fmaxf(red[0][2 * hh], red[0][2 * hh + 1]));
-    float w = 0.f, zl = 0.f;
-    if (live) {  // the tensor-core splits keep their maxima in base 2
-      w = exp2f(v.x - Mn);
-      zl = w * v.y;
-      w *= scv;
-    }
-    if (t64 < nb) wts[t64][hh] = w;
-    zl = warp_sum(zl);
-    if (lane == 0) red[1][warp] = zl;
-    __syncthreads();
-    const float f = M == -INFINITY ? 0.f : exp2f(M - Mn);
-    Z = Z * f + (red[1][2 * hh] + red[1][2 * hh + 1]);
+  for (int k = 0; k < 4; ++k) acc[0][k] = acc[1][k] = 0.f;
+  for (int s0 = 0; s0 < ns; s0 += kGBatch) {
+    float4 v[kGBatch];
+    float2 sc[kGBatch];
+    uint32_t x[kGBatch][4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) acc[k] *= f;
-    M = Mn;
-    ok = __syncthreads_and(mbar_wait(bar, phase)) != 0;
-    phase ^= 1;
-    if (!ok) break;
-    for (int u = 0; u < nb; ++u) {
-      const float wu = wts[u][hh];
-      if (wu > 0.f) {
-        const uint4 r = *reinterpret_cast<const uint4*>(cs_raw + u * kGRow + hh * (kGDim * 2) + 16 * t64);
+    for (int u = 0; u < kGBatch; ++u) {
+      if (s0 + u < ns) {
+        const int64_t slot = base + s0 + u;
+        v[u] = __ldcg(ml + slot * (kGHeads / 2) + hp);
+        sc[u] = __ldcg(scp + slot * (kGHeads / 2) + hp);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[u][k] = __ldcg(ph + (slot * kGDim + d0 + k) * (kGHeads / 2) + hp);
+      } else {
+        v[u] = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kGBatch; ++u) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float m = j ? v[u].z : v[u].x, l = j ? v[u].w : v[u].y;
+        if (!(l > 0.f)) continue;  // l = 0: the split holds no keys (or gave up)
+        if (m > M[j]) {            // a new maximum: rescale what is merged so far
+          const float f = M[j] == -INFINITY ? 0.f : exp2f(M[j] - m);
+          Z[j] *= f;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc[j][k] *= f;
+          M[j] = m;
+        }
+        const float w = exp2f(m - M[j]);
+        Z[j] = fmaf(w, l, Z[j]);
+        const float ws_ = w * (j ? sc[u].y : sc[u].x);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float2 x = half2_bits_to_float2(k == 0 ? r.x : k == 1 ? r.y : k == 2 ? r.z : r.w);
-          acc[2 * k] = fmaf(wu, x.x, acc[2 * k]);
-          acc[2 * k + 1] = fmaf(wu, x.y, acc[2 * k + 1]);
+          const float2 xf = half2_bits_to_float2(x[u][k]);
+          acc[j][k] = fmaf(ws_, j ? xf.y : xf.x, acc[j][k]);
         }
       }
     }
-    __syncthreads();  // the buffer, weights and reductions are reused by the next round
   }
-  if (!ok) {
-    if (tid == 0) atomicOr(status, CKV_DEV_TIMEOUT);
-    mbar_wait(bar, phase ^ 1);  // let this round's copies land before the CTA exits (bounded)
-    o[0] = o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    return;
-  }
-  if (!(Z > 0.f)) {  // no key: a zero output (the rotary table may not have been written)
-    o[0] = o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    return;
-  }
-  const float inv = 1.f / Z;
-  float v8[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) v8[k] = acc[k] * inv;
   const int first_rope = (kGDim - p.d_r) / 2;
   const double* rope = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {  // inverse rotation by the query position
-    const int pr = 4 * t64 + k;
-    if (pr >= first_rope) {
-      const double cs = rope[2 * (pr - first_rope)], sn = rope[2 * (pr - first_rope) + 1];
-      const double a0 = v8[2 * k], e0 = v8[2 * k + 1];
-      v8[2 * k] = static_cast<float>(a0 * cs + e0 * sn);
-      v8[2 * k + 1] = static_cast<float>(e0 * cs - a0 * sn);
+  for (int j = 0; j < 2; ++j) {
+    float4* o = j ? o1 : o0;
+    if (!(Z[j] > 0.f)) {  // no key: a zero output
+      *o = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
     }
+    const float inv = 1.f / Z[j];
+    float v4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v4[k] = acc[j][k] * inv;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {  // inverse rotation by the query position
+      const int pr = d0 / 2 + k;
+      if (pr >= first_rope) {
+        const double cs = rope[2 * (pr - first_rope)], sn = rope[2 * (pr - first_rope) + 1];
+        const double a0 = v4[2 * k], e0 = v4[2 * k + 1];
+        v4[2 * k] = static_cast<float>(a0 * cs + e0 * sn);
+        v4[2 * k + 1] = static_cast<float>(e0 * cs - a0 * sn);
+      }
+    }
+    *o = make_float4(v4[0], v4[1], v4[2], v4[3]);
   }
-  o[0] = make_float4(v8[0], v8[1], v8[2], v8[3]);
-  o[1] = make_float4(v8[4], v8[5], v8[6], v8[7]);
 }
 
 template <int D>
@@ -442,6 +418,8 @@ AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_
   const size_t sc_bytes = align_up(n_slot * sizeof(float), 256);
   const size_t rope_bytes = align_up(static_cast<size_t>(batch) * (p.d_r / 2 + 1) * 2 * sizeof(double), 256);
   w.half_parts = attention_tc_supported(p);
+  const size_t qi_bytes = w.half_parts ? align_up(static_cast<size_t>(batch) * kQImageBytes, 256) : 0;
+  const size_t qs_bytes = w.half_parts ? align_up(static_cast<size_t>(batch) * kQiHeads * sizeof(float), 256) : 0;
   if (base) {
     char* c = static_cast<char*>(base);
     w.part_o = reinterpret_cast<float*>(c);
@@ -449,15 +427,19 @@ AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_
     w.part_ml = reinterpret_cast<float*>(c + o_bytes);
     w.rope = reinterpret_cast<double*>(c + o_bytes + ml_bytes);
     w.part_sc = reinterpret_cast<float*>(c + o_bytes + ml_bytes + rope_bytes);
+    if (w.half_parts) {
+      w.qimage = reinterpret_cast<uint8_t*>(c + o_bytes + ml_bytes + rope_bytes + sc_bytes);
+      w.qscale = reinterpret_cast<float*>(c + o_bytes + ml_bytes + rope_bytes + sc_bytes + qi_bytes);
+    }
   }
-  w.bytes = o_bytes + ml_bytes + rope_bytes + sc_bytes;
+  w.bytes = o_bytes + ml_bytes + rope_bytes + sc_bytes + qi_bytes + qs_bytes;
   return w;
 }
 
 cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq_len,
                              int max_seq_len, const float* q, const int32_t* idx,
                              const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
-                             uint32_t* status, cudaStream_t stream, bool prep_done) {
+                             uint32_t* status, cudaStream_t stream, bool prep_done, bool early) {
   cudaError_t e = cudaSuccess;
   if (!prep_done && !attention_tc_supported(p)) {  // the tensor-core kernel writes the table itself
     e = launch_kernel(attn_prep_kernel, dim3(1, batch), dim3(kPrepThreads), 0, stream, p, seq_len, max_seq_len,
@@ -466,7 +448,8 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
   }
   prof_begin(kProfAttention, stream);
   if (attention_tc_supported(p)) {
-    e = launch_attention_tc(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream, prep_done);
+    e = launch_attention_tc(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream, early,
+                            prep_done);
   } else {
     switch (p.D) {
       case 64: e = launch_simt_d<64>(p, batch, seq_len, max_seq_len, q, idx, cnt, idx_stride, ws, status, stream); break;
@@ -480,12 +463,8 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
   if (e != cudaSuccess) return e;
   dim3 grid(p.H, batch);
   if (ws.half_parts) {   // tensor-core path: H = 64, D = 512
-    const int gs = ws.splits < kGS ? ws.splits : kGS;
-    const int smem = gs * static_cast<int>(kGRow);
-    e = allow_smem(reinterpret_cast<const void*>(attn_combine_tc_kernel), smem);
-    if (e != cudaSuccess) return e;
-    e = launch_kernel(attn_combine_tc_kernel, dim3(p.H / kGH, batch), dim3(kGThreads), smem, stream, p,
-                      seq_len, max_seq_len, cnt, idx != nullptr, idx_stride, gs, ws, out, status);
+    e = launch_kernel(attn_combine_tc_kernel, dim3(kGDim / kGDimsPerCta, batch), dim3(kGThreads), 0, stream, p,
+                      seq_len, max_seq_len, cnt, idx != nullptr, idx_stride, ws, out, status);
   } else {
     const dim3 block(p.D / 2);   // one thread per pair of dims: 32 .. 512
     e = launch_kernel(attn_combine_kernel, grid, block, 0, stream, p, seq_len, max_seq_len, cnt,

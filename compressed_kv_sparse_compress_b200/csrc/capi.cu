@@ -401,7 +401,7 @@ int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int3
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   // append of the token at seq_len[b] - 1 side by side with the query pass (q_bar and the cos/sin
   // table of the rotary pairs), then selection (sparse layers) and attention
-  const QueryPrepOut prep{aw.rope};
+  const QueryPrepOut prep{aw.rope, aw.qimage, aw.qscale};  // the image only for tensor-core layers
   // With more (request, slice) CTAs than SMs the append and the query pass run side by side in one
   // front kernel. With fewer, they stay two kernels: the front kernel's CTAs take a whole SM's
   // registers each, which keeps the next kernel's CTAs from becoming resident early (measured:
@@ -421,10 +421,11 @@ int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int3
     if (e != cudaSuccess) return CKV_ERR_CUDA;
   }
   // the cos/sin table is written when the front kernel ran or the indexer's q-bar pass wrote it
-  // (the tensor-core attention writes it itself either way)
+  // (the tensor-core attention computes it itself either way); the step's first kernel waited for
+  // the producers of q and seq_len, so the attention may read them early
   e = launch_attention(p, batch, d_seq_len, max_seq_len, d_q, top_k > 0 ? d_idx : nullptr,
                        top_k > 0 ? d_cnt : nullptr, top_k > 0 ? top_k : 0, d_out, aw, d_status, s,
-                       front || top_k > 0);
+                       front || top_k > 0, true);
   return e == cudaSuccess ? CKV_OK : CKV_ERR_CUDA;
 }
 

@@ -81,6 +81,20 @@ __device__ __forceinline__ double rope_inv_freq(const LayerParams& p, int i) {
   return i < LayerParams::kRopeTable ? p.inv_freq[i] : rope_inv_freq(i, p.d_r, p.rope_base);
 }
 
+// sin and cos of a rotary angle (fp64, |angle| up to ~2^40): the angle is first reduced by the
+// nearest multiple k of 2 pi with 2 pi split into a head and a tail double (Cody and Waite's
+// additive reduction), so that the library's sincos sees |r| <= pi, its short path. The reduction
+// error is about k * 2^-106, far below the fp64 rounding of the angle itself.
+__device__ __forceinline__ void rope_sincos(double angle, double* sn, double* cs) {
+  constexpr double kTwoPiHi = 6.283185307179586;        // the double nearest 2 pi
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;   // 2 pi - kTwoPiHi
+  constexpr double kInvTwoPi = 0.15915494309189535;
+  const double k = rint(angle * kInvTwoPi);
+  double r = fma(-k, kTwoPiHi, angle);
+  r = fma(-k, kTwoPiLo, r);
+  sincos(r, sn, cs);
+}
+
 // rotate the pair (a, b) by angle pos * inv_freq (inverse: by the negative angle), in fp64
 __device__ __forceinline__ void rope_rotate_pair(double a, double b, double pos, double inv_freq,
                                                  bool inverse, double* oa, double* ob) {

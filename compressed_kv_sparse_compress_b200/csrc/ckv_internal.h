@@ -74,7 +74,9 @@ IndexerWs indexer_ws_layout(void* base, const LayerParams& p, int batch, int max
 // Output of the query pass that the attention of the same layer and step can take over: the
 // cos/sin table of the rotary pairs at the query position (null: not written).
 struct QueryPrepOut {
-  double* rope;
+  double* rope;        // [B][d_r/2 + 1][2] cos, sin of the rotary pairs at the query position
+  uint8_t* qimage;     // [B][128 KB] the tensor-core attention's query operand (qimage.cuh), or null
+  float* qscale;       // [B][64] its per-head power-of-two scales
 };
 // skip_qbar: q_bar, the counts and the reset of the selection state are already done (by the
 // fused step's front kernel)
@@ -119,13 +121,16 @@ cudaError_t launch_mh_indexer(const LayerParams& p, const IndexParams& ip, int b
 // ---------------------------------------------------------------------------- attention
 struct AttnWs {
   float* part_o;     // [B][S][H][D]   un-normalised partial outputs (CUDA-core path)
-  uint16_t* part_h;  // [B][S][H][D]   tensor-core path: fp16 partial outputs divided by part_sc
-                     //                (same memory as part_o)
+  uint16_t* part_h;  // [B][S][D][H]   tensor-core path: fp16 partial outputs, rows of 64 heads per
+                     //                dim, head h divided by part_sc (same memory as part_o)
   float* part_sc;    // [B][S][H]      tensor-core path: power-of-two scale of each partial
   bool half_parts;   // which of the two forms the splits write (the tensor-core form)
   float* part_ml;    // [B][S][H][2]   running max and sum of each split (max in nats on the
                      //                CUDA-core path, in base 2 on the tensor-core path)
   double* rope;      // [B][d_r/2][2]  cos, sin of each rotary pair at the query position
+  uint8_t* qimage;   // [B][128 KB]    tensor-core path: the query operand, written by the step's
+                     //                query pass (qimage.cuh); null for other layers
+  float* qscale;     // [B][64]        its per-head scales
   int splits;        // S: splits per request
   int keys_per_split;
   size_t bytes;
@@ -136,13 +141,16 @@ cudaError_t attention_force_timeout(int request);
 AttnWs attention_ws_layout(void* base, const LayerParams& p, int batch, int max_seq_len,
                            int max_selected);
 
-// prep_done: the cos/sin table is already in ws (written by the indexer's query pass of the same
-// step), so the CUDA-core path launches no prep kernel (the tensor-core kernel writes the table
-// itself)
+// prep_done: the cos/sin table is already in ws (written by the indexer's query pass or the front
+// kernel of the same step), so the CUDA-core path launches no prep kernel (the tensor-core kernel
+// computes the table itself and writes it when it is not there). early: the call is part of a
+// fused decode step whose first kernel has already waited for the producers of q and seq_len, so
+// the tensor-core kernel may read them before waiting for its predecessor.
 cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq_len,
                              int max_seq_len, const float* q, const int32_t* idx,
                              const int32_t* cnt, int idx_stride, float* out, const AttnWs& ws,
-                             uint32_t* status, cudaStream_t stream, bool prep_done = false);
+                             uint32_t* status, cudaStream_t stream, bool prep_done = false,
+                             bool early = false);
 
 // ---------------------------------------------------------------------------- fused step
 // First kernel of ckv_decode_step: the append of the new token (at seq_len[b] - 1) side by side

@@ -141,6 +141,10 @@ __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const
   griddep_launch();
   __shared__ double part[kQbarThreads][2];
   qbar_slice(p, seq_len, max_seq_len, q, ws, status, prep, blockIdx.x, blockIdx.y, threadIdx.x, part, 0);
+  if (prep.qimage) {  // the attention's query image, heads 8 x .. 8 x + 7 (slices = 8)
+    __shared__ double rope_tmp[2 * kQiMaxRopePairs];
+    qimage_part(p, seq_len, max_seq_len, q, prep, blockIdx.x, blockIdx.y, threadIdx.x, rope_tmp, 0);
+  }
 }
 
 // ---------------------------------------------------------------------------- scoring
@@ -777,6 +781,7 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
   const int64_t stride = score_stride(p.r, max_seq_len);
   float* sc = scores ? scores : ws.scores;
   cudaError_t e = cudaSuccess;
+  static_assert(kQbarSlices * 8 == kQiHeads, "one query-image part (8 heads) per q_bar slice");
   if (!skip_qbar) {
     e = launch_kernel(qbar_kernel, dim3(kQbarSlices, batch), dim3(kQbarThreads), 0, stream, p, seq_len,
                       max_seq_len, q, ws, status, prep);

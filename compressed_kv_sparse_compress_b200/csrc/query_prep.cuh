@@ -6,6 +6,7 @@
 #pragma once
 
 #include "ckv_internal.h"
+#include "qimage.cuh"
 
 namespace ckv {
 
@@ -106,6 +107,40 @@ __device__ __forceinline__ void prep_part(const LayerParams& p, const int32_t* s
     rope_g[2 * i] = cs;
     rope_g[2 * i + 1] = sn;
   }
+}
+
+// Per request: the query image of heads 8 part .. 8 part + 7 (qimage.cuh) for the tensor-core
+// attention, one warp per head, by 256 threads with ids tid that synchronise through barrier
+// bar_id; rope_tmp is shared memory for the cos/sin table (2 * d_r/2 doubles). Only for layers of
+// 64 heads of dimension 512 (the caller checks); a bad length leaves the image unwritten.
+__device__ __forceinline__ void qimage_part(const LayerParams& p, const int32_t* seq_len, int max_seq_len,
+                                            const float* q, const QueryPrepOut& prep, int part, int b, int tid,
+                                            double* rope_tmp, int bar_id) {
+  const int L = seq_len[b];
+  if (L < 1 || L > max_seq_len) return;
+  const int w = tid >> 5, lane = tid & 31, h = 8 * part + w;
+  float x[16];
+  const float4* src = reinterpret_cast<const float4*>(q + (static_cast<int64_t>(b) * kQiHeads + h) * kQiDim + 16 * lane);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float4 v = __ldg(src + k);
+    x[4 * k] = v.x;
+    x[4 * k + 1] = v.y;
+    x[4 * k + 2] = v.z;
+    x[4 * k + 3] = v.w;
+  }
+  for (int i = tid; i < p.d_r / 2; i += kPrepThreads)
+    rope_sincos(static_cast<double>(L - 1) * rope_inv_freq(p, i), &rope_tmp[2 * i + 1], &rope_tmp[2 * i]);
+  group_sync(bar_id);
+  uint4 hi[2], lo[2];
+  const float sc = qimage_head(x, lane, (kQiDim - p.d_r) / 2, rope_tmp, hi, lo);
+  uint8_t* img = prep.qimage + static_cast<int64_t>(b) * kQImageBytes;
+  const int rh = qimage_row(h, 0), rl = qimage_row(h, 1);
+  *reinterpret_cast<uint4*>(img + qimage_offset(rh, 2 * lane)) = hi[0];
+  *reinterpret_cast<uint4*>(img + qimage_offset(rh, 2 * lane + 1)) = hi[1];
+  *reinterpret_cast<uint4*>(img + qimage_offset(rl, 2 * lane)) = lo[0];
+  *reinterpret_cast<uint4*>(img + qimage_offset(rl, 2 * lane + 1)) = lo[1];
+  if (lane == 0) prep.qscale[static_cast<int64_t>(b) * kQiHeads + h] = sc;
 }
 
 }  // namespace ckv
