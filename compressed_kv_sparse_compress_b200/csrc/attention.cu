@@ -287,29 +287,34 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u) {
 
 // Merge for the tensor-core path (H = 64, D = 512): split s of request b holds O_s as fp16 rows of 64
 // heads per dim (part_h[b][s][d][h], head h divided by part_sc[b][s][h]) and (m, l) per head with
-// the maximum in base 2. One CTA per (request, block of 32 dims); thread t merges heads 2 (t % 32),
-// 2 (t % 32) + 1 over dims 4 (t / 32) .. 4 (t / 32) + 3 of the block, so that a warp reads 128
-// contiguous bytes per dim. Each thread keeps its own running maximum, sum and accumulators (no
-// barrier), reading the splits' partials and weights from L2 a few splits at a time.
-constexpr int kGThreads = 256;
+// the maximum in base 2. One CTA per (request, block of 16 dims); thread t merges heads
+// 2 (t % 32), 2 (t % 32) + 1 over dims 4 ((t / 32) % 4) .. + 3 of the block (a warp reads 128
+// contiguous bytes per dim) for the splits of its group t / 128: each of the G split groups keeps
+// its own running maximum, sum and accumulators, reading the partials from L2 eight splits at a
+// time, and group 0 merges them in shared memory (log-sum-exp). G = 4 when the requests have many
+// splits, else 1.
 constexpr int kGDim = 512;
 constexpr int kGHeads = 64;
-constexpr int kGDimsPerCta = 32;
-constexpr int kGBatch = 4;  // splits whose loads are in flight together
+constexpr int kGDimsPerCta = 16;
+constexpr int kGBatch = 8;  // splits whose loads are in flight together
 
-__global__ void __launch_bounds__(kGThreads) attn_combine_tc_kernel(
+template <int kGGroups>
+__global__ void __launch_bounds__(128 * kGGroups) attn_combine_tc_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const int32_t* cnt, bool sparse,
     int idx_stride, AttnWs ws, float* out, uint32_t* status) {
   griddep_wait();
   griddep_launch();
+  __shared__ float4 red_acc[kGGroups > 1 ? kGGroups - 1 : 1][128][2];  // groups 1..: the two heads' accumulators
+  __shared__ float4 red_mz[kGGroups > 1 ? kGGroups - 1 : 1][128];      // (M0, Z0, M1, Z1)
   const int blk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int hp = tid & 31, d0 = kGDimsPerCta * blk + 4 * (tid >> 5);
+  const int hp = tid & 31, sg = tid >> 7, tg = tid & 127;
+  const int d0 = kGDimsPerCta * blk + 4 * ((tid >> 5) & 3);
   float4* o0 = reinterpret_cast<float4*>(out + (static_cast<int64_t>(b) * kGHeads + 2 * hp) * kGDim + d0);
   float4* o1 = o0 + kGDim / 4;
   const int L = seq_len[b];
   if (L < 1 || L > max_seq_len) {
     if (blk == 0 && tid == 0) atomicOr(status, CKV_DEV_BAD_LENGTH);
-    *o0 = *o1 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (sg == 0) *o0 = *o1 = make_float4(0.f, 0.f, 0.f, 0.f);
     return;
   }
   const KeyList kl = key_list(p, L, cnt, sparse, idx_stride, b);
@@ -321,7 +326,22 @@ __global__ void __launch_bounds__(kGThreads) attn_combine_tc_kernel(
   float M[2] = {-INFINITY, -INFINITY}, Z[2] = {0.f, 0.f}, acc[2][4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[0][k] = acc[1][k] = 0.f;
-  for (int s0 = 0; s0 < ns; s0 += kGBatch) {
+  // merge (m, l, x) of one split into this thread's running state (j: head of the pair)
+  auto merge = [&](int j, float m, float l, float w_scale, const float (&x)[4]) {
+    if (!(l > 0.f)) return;  // l = 0: the split holds no keys (or gave up)
+    if (m > M[j]) {          // a new maximum: rescale what is merged so far
+      const float f = M[j] == -INFINITY ? 0.f : exp2f(M[j] - m);
+      Z[j] *= f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[j][k] *= f;
+      M[j] = m;
+    }
+    const float w = exp2f(m - M[j]);
+    Z[j] = fmaf(w, l, Z[j]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[j][k] = fmaf(w * w_scale, x[k], acc[j][k]);
+  };
+  for (int s0 = sg * kGBatch; s0 < ns; s0 += kGGroups * kGBatch) {
     float4 v[kGBatch];
     float2 sc[kGBatch];
     uint32_t x[kGBatch][4];
@@ -339,26 +359,42 @@ __global__ void __launch_bounds__(kGThreads) attn_combine_tc_kernel(
     }
 #pragma unroll
     for (int u = 0; u < kGBatch; ++u) {
+      float xa[4], xb[4];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float m = j ? v[u].z : v[u].x, l = j ? v[u].w : v[u].y;
-        if (!(l > 0.f)) continue;  // l = 0: the split holds no keys (or gave up)
-        if (m > M[j]) {            // a new maximum: rescale what is merged so far
-          const float f = M[j] == -INFINITY ? 0.f : exp2f(M[j] - m);
-          Z[j] *= f;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc[j][k] *= f;
-          M[j] = m;
-        }
-        const float w = exp2f(m - M[j]);
-        Z[j] = fmaf(w, l, Z[j]);
-        const float ws_ = w * (j ? sc[u].y : sc[u].x);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 xf = half2_bits_to_float2(x[u][k]);
-          acc[j][k] = fmaf(ws_, j ? xf.y : xf.x, acc[j][k]);
-        }
+      for (int k = 0; k < 4; ++k) {
+        const float2 xf = half2_bits_to_float2(x[u][k]);
+        xa[k] = xf.x;
+        xb[k] = xf.y;
       }
+      merge(0, v[u].x, v[u].y, sc[u].x, xa);
+      merge(1, v[u].z, v[u].w, sc[u].y, xb);
+    }
+  }
+  // groups 1.. hand their state to group 0
+  if (kGGroups > 1 && sg > 0) {
+    red_mz[sg - 1][tg] = make_float4(M[0], Z[0], M[1], Z[1]);
+    red_acc[sg - 1][tg][0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+    red_acc[sg - 1][tg][1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
+  }
+  if (kGGroups > 1) {
+    __syncthreads();
+    if (sg > 0) return;
+  }
+#pragma unroll
+  for (int g = 0; g < kGGroups - 1; ++g) {
+    const float4 mz = red_mz[g][tg];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float m = j ? mz.z : mz.x, z = j ? mz.w : mz.y;
+      if (!(z > 0.f)) continue;
+      const float4 a = red_acc[g][tg][j];
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float Mn = fmaxf(M[j], m);
+      const float f_self = M[j] == -INFINITY ? 0.f : exp2f(M[j] - Mn), f_other = exp2f(m - Mn);
+      Z[j] = Z[j] * f_self + z * f_other;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[j][k] = acc[j][k] * f_self + av[k] * f_other;
+      M[j] = Mn;
     }
   }
   const int first_rope = (kGDim - p.d_r) / 2;
@@ -463,7 +499,10 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
   if (e != cudaSuccess) return e;
   dim3 grid(p.H, batch);
   if (ws.half_parts) {   // tensor-core path: H = 64, D = 512
-    e = launch_kernel(attn_combine_tc_kernel, dim3(kGDim / kGDimsPerCta, batch), dim3(kGThreads), 0, stream, p,
+    // four split groups per CTA when the requests have many splits
+    const bool many = ws.splits > 2 * kGBatch;
+    auto kern = many ? attn_combine_tc_kernel<4> : attn_combine_tc_kernel<1>;
+    e = launch_kernel(kern, dim3(kGDim / kGDimsPerCta, batch), dim3(many ? 512 : 128), 0, stream, p,
                       seq_len, max_seq_len, cnt, idx != nullptr, idx_stride, ws, out, status);
   } else {
     const dim3 block(p.D / 2);   // one thread per pair of dims: 32 .. 512
