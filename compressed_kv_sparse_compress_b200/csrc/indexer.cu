@@ -442,7 +442,9 @@ __global__ void __launch_bounds__(kThreads) topk_mark_kernel(const float* scores
   word |= __shfl_xor_sync(0xffffffffu, word, 2);
   word |= __shfl_xor_sync(0xffffffffu, word, 4);
   if ((lane & 7) == 0 && (w0 + (lane >> 3)) * 32 < N) bm[w0 + (lane >> 3)] = word;
-  // boundary-bin candidates: one atomic per warp, then each lane writes its own
+  // boundary-bin candidates: one atomic per CTA (the request's counter is shared by all its
+  // CTAs), then each lane writes its own
+  __shared__ uint32_t wtot[kWarps + 1];
   const int mine = __popc(cnd);
   int incl = mine;
 #pragma unroll
@@ -450,13 +452,22 @@ __global__ void __launch_bounds__(kThreads) topk_mark_kernel(const float* scores
     const int t = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += t;
   }
-  const int total = __shfl_sync(0xffffffffu, incl, 31);
-  if (total) {
-    uint32_t base = 0;
-    if (lane == 31) base = atomicAdd(ws.cand_cnt + b, static_cast<uint32_t>(total));
-    base = __shfl_sync(0xffffffffu, base, 31);
+  if (lane == 31) wtot[warp] = static_cast<uint32_t>(incl);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t run = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const uint32_t t = wtot[w];
+      wtot[w] = run;
+      run += t;
+    }
+    wtot[kWarps] = run ? atomicAdd(ws.cand_cnt + b, run) : 0u;
+  }
+  __syncthreads();
+  if (mine) {
     uint2* cand = ws.cand + static_cast<int64_t>(b) * stride;
-    uint32_t pos = base + incl - mine;
+    uint32_t pos = wtot[kWarps] + wtot[warp] + static_cast<uint32_t>(incl - mine);
 #pragma unroll
     for (int e = 0; e < 4; ++e)
       if (cnd & (1u << e)) cand[pos++] = make_uint2(keys[e], static_cast<uint32_t>(j + e));
@@ -530,7 +541,16 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, 
     const uint32_t m = ws.cand_cnt[b];
     const uint2* cand = ws.cand + static_cast<int64_t>(b) * stride;
     if (m <= kFinishCandSmem) {
-      for (uint32_t i = threadIdx.x; i < m; i += blockDim.x) cand_s[i] = __ldcg(cand + i);
+      // four loads in flight per thread
+      for (uint32_t i0 = threadIdx.x; i0 < m; i0 += 4 * blockDim.x) {
+        uint2 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (i0 + u * blockDim.x < m) v[u] = __ldcg(cand + i0 + u * blockDim.x);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (i0 + u * blockDim.x < m) cand_s[i0 + u * blockDim.x] = v[u];
+      }
       __syncthreads();
       cand = cand_s;
     }
@@ -571,22 +591,39 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(int top_k, 
     __threadfence_block();
     __syncthreads();
   }
-  // compaction of the bitmap into ascending indices
+  // compaction of the bitmap into ascending indices: thread t takes the words [w0, w1); when they
+  // are at most kRegWords, all their loads are in flight at once and the words stay in registers
+  // for the second pass
+  constexpr int kRegWords = 8;
   const int64_t nw = (N + 31) / 32;
   const int64_t w0 = nw * threadIdx.x / blockDim.x, w1 = nw * (threadIdx.x + 1) / blockDim.x;
+  const bool in_regs = w1 - w0 <= kRegWords;
+  uint32_t wr[kRegWords];
   uint32_t c = 0;
-  for (int64_t w = w0; w < w1; ++w) c += __popc(__ldcg(bm + w));
+  if (in_regs) {
+#pragma unroll
+    for (int i = 0; i < kRegWords; ++i) wr[i] = w0 + i < w1 ? __ldcg(bm + w0 + i) : 0u;
+#pragma unroll
+    for (int i = 0; i < kRegWords; ++i) c += __popc(wr[i]);
+  } else {
+    for (int64_t w = w0; w < w1; ++w) c += __popc(__ldcg(bm + w));
+  }
   const uint32_t incl = block_inclusive_scan<uint32_t>(c, sh, nullptr);
   int64_t pos = incl - c;
   int32_t* out = idx + static_cast<int64_t>(b) * top_k;
-  for (int64_t w = w0; w < w1; ++w) {
-    uint32_t word = __ldcg(bm + w);
+  auto emit = [&](int64_t w, uint32_t word) {
     while (word) {
       const int bit = __ffs(word) - 1;
       word &= word - 1;
       if (pos < top_k) out[pos] = static_cast<int32_t>(w * 32 + bit);
       ++pos;
     }
+  };
+  if (in_regs) {
+#pragma unroll
+    for (int i = 0; i < kRegWords; ++i) emit(w0 + i, wr[i]);
+  } else {
+    for (int64_t w = w0; w < w1; ++w) emit(w, __ldcg(bm + w));
   }
   for (int64_t i = k_eff + threadIdx.x; i < top_k; i += blockDim.x) out[i] = -1;
   if (threadIdx.x == 0) cnt[b] = static_cast<int32_t>(k_eff);
