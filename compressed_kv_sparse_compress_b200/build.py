@@ -11,7 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libckv.so")
-SOURCES = ["capi.cu", "append.cu", "indexer.cu", "index_mh.cu", "score_nvfp4.cu", "attention.cu", "attention_tc.cu",
+SOURCES = ["capi.cu", "append.cu", "indexer.cu", "index_mh.cu", "attention.cu", "attention_tc.cu",
            "noalloc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

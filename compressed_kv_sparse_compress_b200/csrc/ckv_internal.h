@@ -86,12 +86,6 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
                            cudaStream_t stream, QueryPrepOut prep = {nullptr},
                            bool skip_qbar = false);
 
-// Scores of an NVFP4 compressed cache on the tensor cores (D = 512, ratio <= 4); same outputs as
-// the CUDA-core score kernel (scores, candidate counts untouched, first-digit histogram).
-bool score_nvfp4_tc_supported(const LayerParams& p);
-cudaError_t launch_score_nvfp4_tc(const LayerParams& p, int batch, int max_seq_len, const IndexerWs& ws,
-                                  float* scores, int64_t stride, uint32_t* status, cudaStream_t stream);
-
 // Top-k of the scores a score pass wrote, with the candidate counts, the reset selection state
 // and the first-digit histogram in ws (the kernels after the score pass).
 cudaError_t launch_topk(const LayerParams& p, int batch, int max_seq_len, int top_k, const float* scores,

@@ -827,11 +827,7 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
   switch (p.comp_dtype) {
     case CKV_F32: e = dispatch_score<CKV_F32>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
     case CKV_BF16: e = dispatch_score<CKV_BF16>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
-    case CKV_NVFP4:
-      e = score_nvfp4_tc_supported(p)
-              ? launch_score_nvfp4_tc(p, batch, max_seq_len, ws, sc, stride, status, stream)
-              : dispatch_score<CKV_NVFP4>(p, batch, max_seq_len, ws, sc, stride, status, stream);
-      break;
+    case CKV_NVFP4: e = dispatch_score<CKV_NVFP4>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
     default: e = cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;

@@ -1,5 +1,5 @@
-"""The head-averaged indexer over an NVFP4 compressed cache (scored on the tensor cores at D = 512)
-against the oracle, through the C ABI: scores within 1e-5 of the largest, top-k sets by the set
+"""The head-averaged indexer over an NVFP4 compressed cache at D = 512 against the oracle, through
+the C ABI: scores within 1e-5 of the largest, top-k sets by the set
 rule, on batches whose requests switch inside a CTA's range of tiles, ragged last tiles, queries
 of very different magnitudes, and an unmapped block (flagged, its entries score 0)."""
 
