@@ -110,7 +110,7 @@ constexpr uint32_t kOffQs = kOffAlpha + 2 * kH * 4;      // float[64]: query sca
 constexpr uint32_t kOffInvSc = kOffQs + kH * 4;          // float[64]: 1 / (partial scale) per head
 constexpr uint32_t kOffRope = kOffInvSc + kH * 4;        // double[256][2]: cos, sin per rotary pair
 constexpr uint32_t kOffDummy = kOffRope + kMaxRopePairs * 16;  // 512 B: target of the epilogue's warm-up pass
-constexpr uint32_t kOffMisc = kOffDummy + 512;            // int abort; float F
+constexpr uint32_t kOffMisc = kOffDummy + 512;            // int abort
 constexpr uint32_t kOffBar = kOffMisc + 16;              // kNumBars mbarriers
 constexpr uint32_t kOffTmem = kOffBar + 19 * 8;
 constexpr uint32_t kSmemUsed = kOffTmem + 8;
@@ -317,6 +317,24 @@ __device__ __forceinline__ float pow2_ceil(float x) {
   return e >= 255u ? INFINITY : __uint_as_float(e << 23);
 }
 
+// loads of key bytes, each read once: not kept in L1 (which then holds the registers that the
+// kernel spills)
+__device__ __forceinline__ uint2 ldg_stream2(const void* ptr) {
+  uint2 v;
+  asm("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(ptr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_stream1(const void* ptr) {
+  uint32_t v;
+  asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(ptr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_stream_u8(const void* ptr) {
+  uint16_t v;
+  asm("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(v) : "l"(ptr));
+  return v;
+}
+
 // Raw bytes of one 8-element granule of a key: bf16 16 B, FP8 window 8 B, NVFP4 4 B of codes and
 // the e4m3 scale of its 16-element block.
 struct Raw {
@@ -331,17 +349,17 @@ __device__ __forceinline__ Raw load_granule(const LayerParams& p, int64_t row, b
   r.s = 0;
   if (row < 0) return r;
   if (win) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.win_codes + row * p.win_row_bytes) + g);
+    const uint2 v = ldg_stream2(reinterpret_cast<const uint2*>(p.win_codes + row * p.win_row_bytes) + g);
     r.a.x = v.x;
     r.a.y = v.y;
     return r;
   }
   const uint8_t* base = p.comp_codes + row * p.comp_row_bytes;
   if constexpr (CT == CKV_BF16) {
-    r.a = __ldg(reinterpret_cast<const uint4*>(base) + g);
+    r.a = ldg_stream(reinterpret_cast<const uint4*>(base) + g);
   } else {
-    r.a.x = __ldg(reinterpret_cast<const uint32_t*>(base) + g);
-    r.s = __ldg(p.comp_scales + row * (kD / 16) + (g >> 1));
+    r.a.x = ldg_stream1(reinterpret_cast<const uint32_t*>(base) + g);
+    r.s = ldg_stream_u8(p.comp_scales + row * (kD / 16) + (g >> 1));
   }
   return r;
 }
@@ -439,7 +457,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   float* inv_sc = reinterpret_cast<float*>(base + kOffInvSc);
   double* rope_sm = reinterpret_cast<double*>(base + kOffRope);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc);
-  float* f_final = reinterpret_cast<float*>(base + kOffMisc + 4);
   auto bar = [&](int i) { return sb + kOffBar + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffTmem);
 
@@ -467,7 +484,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   if (tid == 0) {
     init_barriers();
     *abort_flag = 0;
-    *f_final = 0.f;
   }
 
   // ---- start-up that reads only the query and the length: the tensor memory, the rotary table
@@ -646,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       } else if (u < t0 - 2) {
         pv = true;   // tiles t0, t0 + 1 write the P stages of tiles t0 - 4, t0 - 3
       } else {       // either: the output product when its weights are already written
-        pv = !dry && __all_sync(0xffffffffu, mbar_try_wait(bar(kBarPfull + (u & (kPStages - 1))), static_cast<uint32_t>(u >> 2) & 1u));
+        pv = !dry && __all_sync(0xffffffffu, mbar_test_wait(bar(kBarPfull + (u & (kPStages - 1))), static_cast<uint32_t>(u >> 2) & 1u));
       }
       if (pv) {
         const int x = u & (kXStages - 1);
@@ -840,7 +856,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           reinterpret_cast<float2*>(ws.part_ml)[slot + h] = make_float2(m_run, l);
           ws.part_sc[slot + h] = sc * F_run;
         }
-        if (h == 0) *f_final = F_run;
       }
     }
   } else {
@@ -976,7 +991,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     if (tid == 0) {
       for (int i = 0; i < kNumBars; ++i) mbar_inval(bar(i));
       init_barriers();
-      *f_final = 0.f;
     }
     __syncthreads();
     tc_fence_after();
@@ -989,6 +1003,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
+    if (prepared) mbar_wait(bar(kBarQfull), 0);  // no copy in flight at the exit (also after an abort)
     tc_fence_after();
     tmem_dealloc(*tmem_slot, kTmemCols);
   }
