@@ -289,36 +289,61 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u) {
 // heads per dim (part_h[b][s][d][h], head h divided by part_sc[b][s][h]) and (m, l) per head with
 // the maximum in base 2. One CTA per (request, block of 16 dims); thread t merges heads
 // 2 (t % 32), 2 (t % 32) + 1 over dims 4 ((t / 32) % 4) .. + 3 of the block (a warp reads 128
-// contiguous bytes per dim) for the splits of its group t / 128: each of the G split groups keeps
-// its own running maximum, sum and accumulators, reading the partials from L2 eight splits at a
-// time, and group 0 merges them in shared memory (log-sum-exp). G = 4 when the requests have many
-// splits, else 1.
+// contiguous bytes per dim) for the splits of its group g = t / 128 (splits g, g + G, g + 2 G, ..):
+// each of the G split groups keeps its own running maximum, sum and accumulators, reading the
+// partials from L2 kBatch splits at a time, and group 0 merges them in shared memory (log-sum-exp).
+// G = 4 when the requests have more than 16 splits, else 1.
+//
+// The length, the selection count and (rope_ready: written by a kernel before the attention) the
+// cos/sin table are read before the wait: this kernel starts only once every attention CTA that
+// holds keys has passed its own wait, which in turn follows the kernels that wrote them.
 constexpr int kGDim = 512;
 constexpr int kGHeads = 64;
 constexpr int kGDimsPerCta = 16;
-constexpr int kGBatch = 8;  // splits whose loads are in flight together
+constexpr int kGBatch = 8;       // splits whose loads are in flight together (one group)
+constexpr int kGBatchMany = 9;   // the same, per group of four
 
-template <int kGGroups>
+template <int kGGroups, int kBatch>
 __global__ void __launch_bounds__(128 * kGGroups) attn_combine_tc_kernel(
     LayerParams p, const int32_t* seq_len, int max_seq_len, const int32_t* cnt, bool sparse,
-    int idx_stride, AttnWs ws, float* out, uint32_t* status) {
-  griddep_wait();
-  griddep_launch();
+    int idx_stride, AttnWs ws, float* out, uint32_t* status, bool rope_ready) {
   __shared__ float4 red_acc[kGGroups > 1 ? kGGroups - 1 : 1][128][2];  // groups 1..: the two heads' accumulators
   __shared__ float4 red_mz[kGGroups > 1 ? kGGroups - 1 : 1][128];      // (M0, Z0, M1, Z1)
   const int blk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int hp = tid & 31, sg = tid >> 7, tg = tid & 127;
   const int d0 = kGDimsPerCta * blk + 4 * ((tid >> 5) & 3);
+  const int L = __ldcg(seq_len + b);
+  const bool live = L >= 1 && L <= max_seq_len;
+  const int sel = live && sparse ? __ldcg(cnt + b) : 0;
+  // cos, sin of the rotary pairs d0 / 2, d0 / 2 + 1 (inverse rotation of group 0's outputs)
+  const int first_rope = (kGDim - p.d_r) / 2;
+  const double* rope = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
+  double cs[2] = {1.0, 1.0}, sn[2] = {0.0, 0.0};
+  auto load_rope = [&]() {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int pr = d0 / 2 + k;
+      if (pr >= first_rope) {
+        cs[k] = __ldcg(rope + 2 * (pr - first_rope));
+        sn[k] = __ldcg(rope + 2 * (pr - first_rope) + 1);
+      }
+    }
+  };
+  if (rope_ready && live && sg == 0) load_rope();
+  griddep_wait();
+  griddep_launch();
   float4* o0 = reinterpret_cast<float4*>(out + (static_cast<int64_t>(b) * kGHeads + 2 * hp) * kGDim + d0);
   float4* o1 = o0 + kGDim / 4;
-  const int L = seq_len[b];
-  if (L < 1 || L > max_seq_len) {
+  if (!live) {
     if (blk == 0 && tid == 0) atomicOr(status, CKV_DEV_BAD_LENGTH);
     if (sg == 0) *o0 = *o1 = make_float4(0.f, 0.f, 0.f, 0.f);
     return;
   }
-  const KeyList kl = key_list(p, L, cnt, sparse, idx_stride, b);
-  const int ns = static_cast<int>((kl.n_keys + ws.keys_per_split - 1) / ws.keys_per_split);
+  if (!rope_ready && sg == 0) load_rope();
+  const int64_t n_c = L / p.r;
+  const int64_t n_keys = (sparse ? min(static_cast<int64_t>(max(sel, 0)), static_cast<int64_t>(idx_stride)) : n_c) +
+                         min(p.W, L);
+  const int ns = static_cast<int>((n_keys + ws.keys_per_split - 1) / ws.keys_per_split);
   const int64_t base = static_cast<int64_t>(b) * ws.splits;
   const float4* ml = reinterpret_cast<const float4*>(ws.part_ml);           // (m, l) of 2 heads
   const float2* scp = reinterpret_cast<const float2*>(ws.part_sc);          // scales of 2 heads
@@ -341,14 +366,15 @@ __global__ void __launch_bounds__(128 * kGGroups) attn_combine_tc_kernel(
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[j][k] = fmaf(w * w_scale, x[k], acc[j][k]);
   };
-  for (int s0 = sg * kGBatch; s0 < ns; s0 += kGGroups * kGBatch) {
-    float4 v[kGBatch];
-    float2 sc[kGBatch];
-    uint32_t x[kGBatch][4];
+  for (int i0 = 0; sg + kGGroups * i0 < ns; i0 += kBatch) {
+    float4 v[kBatch];
+    float2 sc[kBatch];
+    uint32_t x[kBatch][4];
 #pragma unroll
-    for (int u = 0; u < kGBatch; ++u) {
-      if (s0 + u < ns) {
-        const int64_t slot = base + s0 + u;
+    for (int u = 0; u < kBatch; ++u) {
+      const int s = sg + kGGroups * (i0 + u);
+      if (s < ns) {
+        const int64_t slot = base + s;
         v[u] = __ldcg(ml + slot * (kGHeads / 2) + hp);
         sc[u] = __ldcg(scp + slot * (kGHeads / 2) + hp);
 #pragma unroll
@@ -358,7 +384,7 @@ __global__ void __launch_bounds__(128 * kGGroups) attn_combine_tc_kernel(
       }
     }
 #pragma unroll
-    for (int u = 0; u < kGBatch; ++u) {
+    for (int u = 0; u < kBatch; ++u) {
       float xa[4], xb[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -397,8 +423,6 @@ __global__ void __launch_bounds__(128 * kGGroups) attn_combine_tc_kernel(
       M[j] = Mn;
     }
   }
-  const int first_rope = (kGDim - p.d_r) / 2;
-  const double* rope = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     float4* o = j ? o1 : o0;
@@ -412,12 +436,10 @@ __global__ void __launch_bounds__(128 * kGGroups) attn_combine_tc_kernel(
     for (int k = 0; k < 4; ++k) v4[k] = acc[j][k] * inv;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {  // inverse rotation by the query position
-      const int pr = d0 / 2 + k;
-      if (pr >= first_rope) {
-        const double cs = rope[2 * (pr - first_rope)], sn = rope[2 * (pr - first_rope) + 1];
+      if (d0 / 2 + k >= first_rope) {
         const double a0 = v4[2 * k], e0 = v4[2 * k + 1];
-        v4[2 * k] = static_cast<float>(a0 * cs + e0 * sn);
-        v4[2 * k + 1] = static_cast<float>(e0 * cs - a0 * sn);
+        v4[2 * k] = static_cast<float>(a0 * cs[k] + e0 * sn[k]);
+        v4[2 * k + 1] = static_cast<float>(e0 * cs[k] - a0 * sn[k]);
       }
     }
     *o = make_float4(v4[0], v4[1], v4[2], v4[3]);
@@ -499,11 +521,12 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
   if (e != cudaSuccess) return e;
   dim3 grid(p.H, batch);
   if (ws.half_parts) {   // tensor-core path: H = 64, D = 512
-    // four split groups per CTA when the requests have many splits
+    // four split groups per CTA when the requests have many splits (with fewer, most of the
+    // groups would idle in the CTAs of short requests)
     const bool many = ws.splits > 2 * kGBatch;
-    auto kern = many ? attn_combine_tc_kernel<4> : attn_combine_tc_kernel<1>;
+    auto kern = many ? attn_combine_tc_kernel<4, kGBatchMany> : attn_combine_tc_kernel<1, kGBatch>;
     e = launch_kernel(kern, dim3(kGDim / kGDimsPerCta, batch), dim3(many ? 512 : 128), 0, stream, p,
-                      seq_len, max_seq_len, cnt, idx != nullptr, idx_stride, ws, out, status);
+                      seq_len, max_seq_len, cnt, idx != nullptr, idx_stride, ws, out, status, prep_done);
   } else {
     const dim3 block(p.D / 2);   // one thread per pair of dims: 32 .. 512
     e = launch_kernel(attn_combine_kernel, grid, block, 0, stream, p, seq_len, max_seq_len, cnt,
