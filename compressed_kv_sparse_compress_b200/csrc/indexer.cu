@@ -191,12 +191,16 @@ __device__ __forceinline__ float vec_dot(const float* qv, uint4 raw, uint32_t sc
 }
 
 // NV: 16-byte code vectors per entry (a power of two); U: entries per lane group per chunk
+// Before its wait for the previous kernel (the query pass) the kernel takes the candidate counts
+// from the lengths (the query pass derives the same ones for the selection), partitions the
+// chunks, resolves each warp's first chunk through the block tables and prefetches its entries into
+// L2: the lengths and the block tables come from before the step and no kernel of the step writes
+// them, while the entries (the step's append may complete one) are loaded only after the wait; a
+// prefetch moves no data into registers, so a line the append writes later is read afresh.
 template <int DT, int NV, int U>
-__global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int batch, IndexerWs ws,
-                                                         float* scores, int64_t stride,
-                                                         uint32_t* status) {
-  griddep_wait();
-  griddep_launch();
+__global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int batch, const int32_t* seq_len,
+                                                         int max_seq_len, IndexerWs ws, float* scores,
+                                                         int64_t stride, uint32_t* status) {
   constexpr int LPE = NV < 32 ? NV : 32;  // lanes per entry
   constexpr int VPL = NV / LPE;           // vectors per lane per entry
   constexpr int EPP = 32 / LPE;           // entries per warp pass
@@ -208,10 +212,14 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int b
   int32_t* n_c = chunk_prefix + batch + 1;
   __shared__ int32_t scan_sh[32];
   // chunks per request, exclusive prefix over the batch (one warp when the batch fits it)
+  auto count = [&](int bb) {
+    const int32_t L = __ldcg(seq_len + bb);
+    return L >= 1 && L <= max_seq_len ? L / p.r : 0;
+  };
   if (batch <= 32) {
     if (threadIdx.x < 32) {
       const int bb = threadIdx.x;
-      const int32_t n = bb < batch ? ws.n_c[bb] : 0;
+      const int32_t n = bb < batch ? count(bb) : 0;
       const int32_t s = (n + CH - 1) / CH;
       int32_t incl = s;
 #pragma unroll
@@ -232,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int b
     for (int i = 0; i < per; ++i) {
       const int bb = threadIdx.x * per + i;
       if (bb < batch) {
-        const int32_t n = ws.n_c[bb];
+        const int32_t n = count(bb);
         n_c[bb] = n;
         s += (n + CH - 1) / CH;
       }
@@ -286,7 +294,22 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(LayerParams p, int b
   int cur_b = -1;
   float qreg[VPL][EPV];
   Chunk cur;
-  if (c_lo + warp < c_hi) cur = resolve(c_lo + warp);
+  if (c_lo + warp < c_hi) {
+    cur = resolve(c_lo + warp);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t row = cur.row[u];
+      if (row < 0) continue;
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) {
+        const int v = sub + LPE * k;
+        if ((v & 7) == 0) prefetch_l2(p.comp_codes + row * p.comp_row_bytes + v * 16);  // one per 128-byte line
+      }
+      if (DT == CKV_NVFP4 && sub == 0) prefetch_l2(p.comp_scales + row * sc_bytes);
+    }
+  }
+  griddep_wait();
+  griddep_launch();
   for (int64_t ch = c_lo + warp; ch < c_hi; ch += kWarps) {
     const int b = cur.b;
     if (b != cur_b) {
@@ -759,8 +782,9 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(const float* 
 }
 
 template <int DT, int NV, int U>
-cudaError_t launch_score(const LayerParams& p, int batch, int max_seq_len, const IndexerWs& ws,
-                         float* scores, int64_t stride, uint32_t* status, cudaStream_t stream) {
+cudaError_t launch_score(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
+                         const IndexerWs& ws, float* scores, int64_t stride, uint32_t* status,
+                         cudaStream_t stream) {
   constexpr int LPE = NV < 32 ? NV : 32;
   constexpr int CH = U * (32 / LPE);
   const int64_t per_req = (static_cast<int64_t>(max_seq_len) / p.r + CH - 1) / CH;
@@ -778,15 +802,16 @@ cudaError_t launch_score(const LayerParams& p, int batch, int max_seq_len, const
   if (grid > useful) grid = useful;
   if (grid < 1) grid = 1;
   prof_begin(kProfScore, stream);
-  e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, p, batch, ws,
-                    scores, stride, status);
+  e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, p, batch, seq_len,
+                    max_seq_len, ws, scores, stride, status);
   prof_end(kProfScore, stream);
   return e;
 }
 
 template <int DT>
-cudaError_t dispatch_score(const LayerParams& p, int batch, int max_seq_len, const IndexerWs& ws,
-                           float* scores, int64_t stride, uint32_t* status, cudaStream_t stream) {
+cudaError_t dispatch_score(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
+                           const IndexerWs& ws, float* scores, int64_t stride, uint32_t* status,
+                           cudaStream_t stream) {
   // 16-byte vectors per entry for D = 64 .. 1024: f32 D/4, bf16 D/8, nvfp4 D/32
   const int nv = p.comp_row_bytes / 16;
   constexpr int kMin = DT == CKV_F32 ? 16 : DT == CKV_BF16 ? 8 : 2;
@@ -796,7 +821,7 @@ cudaError_t dispatch_score(const LayerParams& p, int batch, int max_seq_len, con
   case kMin * M:                                                                             \
     return launch_score<DT, kMin * M,                                                        \
                         (kMin * M < 8 ? kMin * M : (kMin * M > 64 ? 512 / (kMin * M) : 8))>( \
-        p, batch, max_seq_len, ws, scores, stride, status, stream);
+        p, batch, seq_len, max_seq_len, ws, scores, stride, status, stream);
   switch (nv) {
     CKV_SCORE_CASE(1)
     CKV_SCORE_CASE(2)
@@ -825,9 +850,9 @@ cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_l
     if (e != cudaSuccess) return e;
   }
   switch (p.comp_dtype) {
-    case CKV_F32: e = dispatch_score<CKV_F32>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
-    case CKV_BF16: e = dispatch_score<CKV_BF16>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
-    case CKV_NVFP4: e = dispatch_score<CKV_NVFP4>(p, batch, max_seq_len, ws, sc, stride, status, stream); break;
+    case CKV_F32: e = dispatch_score<CKV_F32>(p, batch, seq_len, max_seq_len, ws, sc, stride, status, stream); break;
+    case CKV_BF16: e = dispatch_score<CKV_BF16>(p, batch, seq_len, max_seq_len, ws, sc, stride, status, stream); break;
+    case CKV_NVFP4: e = dispatch_score<CKV_NVFP4>(p, batch, seq_len, max_seq_len, ws, sc, stride, status, stream); break;
     default: e = cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
