@@ -417,7 +417,7 @@ int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int3
   if (e != cudaSuccess) return CKV_ERR_CUDA;
   if (top_k > 0) {
     e = launch_indexer(p, batch, d_seq_len, max_seq_len, d_q, top_k, d_idx, d_cnt, nullptr, iw, d_status, s,
-                       prep, front);
+                       prep, front, !front);
     if (e != cudaSuccess) return CKV_ERR_CUDA;
   }
   // the cos/sin table is written when the front kernel ran or the indexer's q-bar pass wrote it

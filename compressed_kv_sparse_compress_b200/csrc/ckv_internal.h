@@ -79,12 +79,13 @@ struct QueryPrepOut {
   float* qscale;       // [B][64] its per-head power-of-two scales
 };
 // skip_qbar: q_bar, the counts and the reset of the selection state are already done (by the
-// fused step's front kernel)
+// fused step's front kernel); early_qbar: the q_bar pass follows the fused step's append, which
+// has waited for the producers of q and the lengths, and may run beside it (qbar_kernel)
 cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
                            int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
                            float* scores, const IndexerWs& ws, uint32_t* status,
                            cudaStream_t stream, QueryPrepOut prep = {nullptr},
-                           bool skip_qbar = false);
+                           bool skip_qbar = false, bool early_qbar = false);
 
 // Top-k of the scores a score pass wrote, with the candidate counts, the reset selection state
 // and the first-digit histogram in ws (the kernels after the score pass).

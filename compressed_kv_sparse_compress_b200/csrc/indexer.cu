@@ -133,11 +133,15 @@ __device__ void find_boundary(const uint32_t* h, int nbins, uint32_t need, bool 
 // ---------------------------------------------------------------------------- q_bar
 
 // q_bar of one slice of one request: qbar_slice (query_prep.cuh).
+// early: the call is part of a fused decode step whose first kernel (the append, which this pass
+// follows) has already waited for the producers of q and the lengths, and nothing this pass reads
+// or writes is touched by the append: the pass runs beside the append and waits for it only before
+// it exits, so that its completion still implies the append's.
 __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const int32_t* seq_len,
                                                             int max_seq_len, const float* q,
                                                             IndexerWs ws, uint32_t* status,
-                                                            QueryPrepOut prep) {
-  griddep_wait();
+                                                            QueryPrepOut prep, bool early) {
+  if (!early) griddep_wait();
   griddep_launch();
   __shared__ double part[kQbarThreads][2];
   qbar_slice(p, seq_len, max_seq_len, q, ws, status, prep, blockIdx.x, blockIdx.y, threadIdx.x, part, 0);
@@ -145,6 +149,7 @@ __global__ void __launch_bounds__(kQbarThreads) qbar_kernel(LayerParams p, const
     __shared__ double rope_tmp[2 * kQiMaxRopePairs];
     qimage_part(p, seq_len, max_seq_len, q, prep, blockIdx.x, blockIdx.y, threadIdx.x, rope_tmp, 0);
   }
+  if (early) griddep_wait();
 }
 
 // ---------------------------------------------------------------------------- scoring
@@ -839,14 +844,14 @@ cudaError_t dispatch_score(const LayerParams& p, int batch, const int32_t* seq_l
 cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
                            int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
                            float* scores, const IndexerWs& ws, uint32_t* status,
-                           cudaStream_t stream, QueryPrepOut prep, bool skip_qbar) {
+                           cudaStream_t stream, QueryPrepOut prep, bool skip_qbar, bool early_qbar) {
   const int64_t stride = score_stride(p.r, max_seq_len);
   float* sc = scores ? scores : ws.scores;
   cudaError_t e = cudaSuccess;
   static_assert(kQbarSlices * 8 == kQiHeads, "one query-image part (8 heads) per q_bar slice");
   if (!skip_qbar) {
     e = launch_kernel(qbar_kernel, dim3(kQbarSlices, batch), dim3(kQbarThreads), 0, stream, p, seq_len,
-                      max_seq_len, q, ws, status, prep);
+                      max_seq_len, q, ws, status, prep, early_qbar);
     if (e != cudaSuccess) return e;
   }
   switch (p.comp_dtype) {
