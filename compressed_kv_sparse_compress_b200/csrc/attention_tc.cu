@@ -1034,7 +1034,9 @@ bool attention_tc_supported(const LayerParams& p) {
 }
 
 // Keys per split: t tiles of 32 keys, t in 1 .. 16, minimising (waves of one CTA per SM) x
-// (t + 2), the 2 standing for a split's fixed cost (start-up, rows, partial write).
+// (t + 8), the 8 standing for a split's fixed cost in tiles (start-up from a cold instruction
+// cache, key resolution, the partial write; measured on the 64-request mixed step: a cost of 2
+// gave 260.5 us per step, 8 to 16 gave 252.7; single-wave launches choose the same t either way).
 int attention_tc_keys_per_split(int batch, int64_t max_keys) {
   const int64_t tiles = max_keys > 0 ? (max_keys + kTile - 1) / kTile : 1;
   const int64_t sms = sm_count();
@@ -1042,7 +1044,7 @@ int attention_tc_keys_per_split(int batch, int64_t max_keys) {
   int64_t best = -1;
   for (int t = 1; t <= kMaxTiles; ++t) {
     const int64_t ctas = static_cast<int64_t>(batch) * ((tiles + t - 1) / t);
-    const int64_t cost = ((ctas + sms - 1) / sms) * (t + 2);
+    const int64_t cost = ((ctas + sms - 1) / sms) * (t + 8);
     if (best < 0 || cost < best) {
       best = cost;
       best_t = t;
