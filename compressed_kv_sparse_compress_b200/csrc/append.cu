@@ -533,29 +533,19 @@ __global__ void __launch_bounds__(kAppendThreads) window_replay_kernel(AppendArg
 
 // ---------------------------------------------------------------------------- fused step front
 
-// First kernel of a fused decode step: the append of one slice (threads 0..255) and, on the other
-// 256 threads, the query pass of the same step (q_bar and the cos/sin table of the rotary pairs on
-// sparse layers, the table alone on dense ones), which reads only the query. The two halves
-// synchronise on barriers 1 and 2 and never wait for each other.
-template <bool kSparse>
+// First kernel of a fused decode step on a dense layer: the append of one slice (threads 0..255)
+// and, on the other 256 threads, the attention's query preparation of the same step (the cos/sin
+// table of the rotary pairs and, for the tensor-core path, the query image), which reads only the
+// query. The two halves synchronise on barriers 1 and 2 and never wait for each other.
 __global__ void __launch_bounds__(2 * kAppendThreads, 1) step_front_kernel(
-    AppendArgs a, int app_slices, const float* q, IndexerWs iws, QueryPrepOut prep, AttnWs aws,
-    int prep_parts) {
+    AppendArgs a, int app_slices, const float* q, QueryPrepOut prep, AttnWs aws, int prep_parts) {
   griddep_wait();
   griddep_launch();
   __shared__ AppendDecodeSmem sm;
-  __shared__ double qsm[512];  // q_bar partial sums [256][2]
   __shared__ double rope_tmp[2 * kQiMaxRopePairs];
   const int x = blockIdx.x, b = blockIdx.y;
   if (threadIdx.x < kAppendThreads) {
     if (x < app_slices) append_decode_slice(a, x, b, threadIdx.x, 1, sm);
-  } else if (kSparse) {
-    if (x < kQbarSlices) {
-      qbar_slice(a.p, a.prev_len, a.max_seq_len, q, iws, a.status, prep, x, b, threadIdx.x - kAppendThreads,
-                 reinterpret_cast<double(*)[2]>(qsm), 2);
-      if (prep.qimage)  // the attention's query image, heads 8 x .. 8 x + 7
-        qimage_part(a.p, a.prev_len, a.max_seq_len, q, prep, x, b, threadIdx.x - kAppendThreads, rope_tmp, 2);
-    }
   } else if (x < prep_parts) {
     prep_part(a.p, a.prev_len, a.max_seq_len, aws, x, b, threadIdx.x - kAppendThreads);
     if (prep.qimage)
@@ -566,20 +556,15 @@ __global__ void __launch_bounds__(2 * kAppendThreads, 1) step_front_kernel(
 }  // namespace
 
 cudaError_t launch_step_front(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
-                              const float* kv_new, const float* logit_new, const float* q, bool sparse,
-                              const IndexerWs& iws, QueryPrepOut prep, const AttnWs& aws,
-                              uint32_t* status, cudaStream_t stream) {
+                              const float* kv_new, const float* logit_new, const float* q,
+                              QueryPrepOut prep, const AttnWs& aws, uint32_t* status, cudaStream_t stream) {
   // the new token of request b is at position seq_len[b] - 1
   const AppendArgs a{p, seq_len, nullptr, max_seq_len, kv_new, logit_new, status, -1};
   const int app_slices = p.D / 2 < kSlicePairs ? 1 : p.D / 2 / kSlicePairs;
   const int prep_parts = prep.qimage ? kQiHeads / 8 : 1;  // the rotary table; the query image by 8 heads
-  const int other = sparse ? kQbarSlices : prep_parts;
-  const dim3 grid(app_slices > other ? app_slices : other, batch);
-  if (sparse)
-    return launch_kernel(step_front_kernel<true>, grid, dim3(2 * kAppendThreads), 0, stream, a, app_slices, q,
-                         iws, prep, aws, prep_parts);
-  return launch_kernel(step_front_kernel<false>, grid, dim3(2 * kAppendThreads), 0, stream, a, app_slices, q,
-                       iws, prep, aws, prep_parts);
+  const dim3 grid(app_slices > prep_parts ? app_slices : prep_parts, batch);
+  return launch_kernel(step_front_kernel, grid, dim3(2 * kAppendThreads), 0, stream, a, app_slices, q, prep, aws,
+                       prep_parts);
 }
 
 cudaError_t launch_append(const LayerParams& p, int batch, const int32_t* prev_len,

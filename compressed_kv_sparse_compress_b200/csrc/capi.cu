@@ -399,25 +399,29 @@ int ckv_decode_step(const ckv_layer_cfg* cfg, const ckv_layer_cache* cache, int3
   AttnWs aw{};
   if (ws_bytes < step_ws_bytes(p, batch, max_seq_len, top_k, &iw, &aw, d_ws)) return CKV_ERR_WORKSPACE;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // append of the token at seq_len[b] - 1 side by side with the query pass (q_bar and the cos/sin
-  // table of the rotary pairs), then selection (sparse layers) and attention
+  // append of the token at seq_len[b] - 1 beside the query pass (q_bar and the cos/sin table of the
+  // rotary pairs on sparse layers, the attention's query preparation on dense ones), then selection
+  // (sparse layers) and attention
   const QueryPrepOut prep{aw.rope, aw.qimage, aw.qscale};  // the image only for tensor-core layers
-  // With more (request, slice) CTAs than SMs the append and the query pass run side by side in one
-  // front kernel. With fewer, they stay two kernels: the front kernel's CTAs take a whole SM's
-  // registers each, which keeps the next kernel's CTAs from becoming resident early (measured:
-  // 57.5 against 54.2 us per step at batch 8, 252.9 against 256.4 us at batch 64).
-  const bool front = static_cast<int64_t>(batch) * 8 > sm_count();
+  // Sparse layers keep the append and the q-bar pass as two kernels, the pass running beside the
+  // append (qbar_kernel, early) and its CTAs leaving room for the next kernel's to become resident.
+  // Dense layers with more (request, slice) CTAs than SMs run the append and the attention's query
+  // preparation side by side in one front kernel; with fewer, the attention prepares its query
+  // itself. Measured (us per step): at batch 8 sparse, 54.2 with two kernels against 57.5 with the
+  // front kernel (before the pass ran beside the append); the 64-request mixed step (a sparse and a
+  // dense layer) 248.9 against 253.5 with the front kernel for both layers; HCA 128K at batch 32,
+  // 49.3 with the front kernel against 56.9 without.
+  const bool front = top_k <= 0 && static_cast<int64_t>(batch) * 8 > sm_count();
   cudaError_t e = cudaSuccess;
   if (front) {
-    e = launch_step_front(p, batch, d_seq_len, max_seq_len, d_kv_new, d_logit_new, d_q, top_k > 0, iw, prep, aw,
-                          d_status, s);
+    e = launch_step_front(p, batch, d_seq_len, max_seq_len, d_kv_new, d_logit_new, d_q, prep, aw, d_status, s);
   } else {
     e = launch_append(p, batch, d_seq_len, nullptr, 1, max_seq_len, d_kv_new, d_logit_new, d_status, s, -1);
   }
   if (e != cudaSuccess) return CKV_ERR_CUDA;
   if (top_k > 0) {
     e = launch_indexer(p, batch, d_seq_len, max_seq_len, d_q, top_k, d_idx, d_cnt, nullptr, iw, d_status, s,
-                       prep, front, !front);
+                       prep, true);
     if (e != cudaSuccess) return CKV_ERR_CUDA;
   }
   // the cos/sin table is written when the front kernel ran or the indexer's q-bar pass wrote it

@@ -78,14 +78,12 @@ struct QueryPrepOut {
   uint8_t* qimage;     // [B][128 KB] the tensor-core attention's query operand (qimage.cuh), or null
   float* qscale;       // [B][64] its per-head power-of-two scales
 };
-// skip_qbar: q_bar, the counts and the reset of the selection state are already done (by the
-// fused step's front kernel); early_qbar: the q_bar pass follows the fused step's append, which
-// has waited for the producers of q and the lengths, and may run beside it (qbar_kernel)
+// early_qbar: the q_bar pass follows the fused step's append, which has waited for the producers
+// of q and the lengths, and may run beside it (qbar_kernel)
 cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
                            int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
                            float* scores, const IndexerWs& ws, uint32_t* status,
-                           cudaStream_t stream, QueryPrepOut prep = {nullptr},
-                           bool skip_qbar = false, bool early_qbar = false);
+                           cudaStream_t stream, QueryPrepOut prep = {nullptr}, bool early_qbar = false);
 
 // Top-k of the scores a score pass wrote, with the candidate counts, the reset selection state
 // and the first-digit histogram in ws (the kernels after the score pass).
@@ -148,12 +146,10 @@ cudaError_t launch_attention(const LayerParams& p, int batch, const int32_t* seq
                              bool early = false);
 
 // ---------------------------------------------------------------------------- fused step
-// First kernel of ckv_decode_step: the append of the new token (at seq_len[b] - 1) side by side
-// with the query pass (q_bar and the query preparation on sparse layers, the preparation alone on
-// dense ones).
+// First kernel of ckv_decode_step on a dense layer: the append of the new token (at seq_len[b] - 1)
+// side by side with the attention's query preparation (the cos/sin table and the query image).
 cudaError_t launch_step_front(const LayerParams& p, int batch, const int32_t* seq_len, int max_seq_len,
-                              const float* kv_new, const float* logit_new, const float* q, bool sparse,
-                              const IndexerWs& iws, QueryPrepOut prep, const AttnWs& aws,
-                              uint32_t* status, cudaStream_t stream);
+                              const float* kv_new, const float* logit_new, const float* q,
+                              QueryPrepOut prep, const AttnWs& aws, uint32_t* status, cudaStream_t stream);
 
 }  // namespace ckv

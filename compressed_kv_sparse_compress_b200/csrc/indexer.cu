@@ -844,16 +844,14 @@ cudaError_t dispatch_score(const LayerParams& p, int batch, const int32_t* seq_l
 cudaError_t launch_indexer(const LayerParams& p, int batch, const int32_t* seq_len,
                            int max_seq_len, const float* q, int top_k, int32_t* idx, int32_t* cnt,
                            float* scores, const IndexerWs& ws, uint32_t* status,
-                           cudaStream_t stream, QueryPrepOut prep, bool skip_qbar, bool early_qbar) {
+                           cudaStream_t stream, QueryPrepOut prep, bool early_qbar) {
   const int64_t stride = score_stride(p.r, max_seq_len);
   float* sc = scores ? scores : ws.scores;
   cudaError_t e = cudaSuccess;
   static_assert(kQbarSlices * 8 == kQiHeads, "one query-image part (8 heads) per q_bar slice");
-  if (!skip_qbar) {
-    e = launch_kernel(qbar_kernel, dim3(kQbarSlices, batch), dim3(kQbarThreads), 0, stream, p, seq_len,
-                      max_seq_len, q, ws, status, prep, early_qbar);
-    if (e != cudaSuccess) return e;
-  }
+  e = launch_kernel(qbar_kernel, dim3(kQbarSlices, batch), dim3(kQbarThreads), 0, stream, p, seq_len,
+                    max_seq_len, q, ws, status, prep, early_qbar);
+  if (e != cudaSuccess) return e;
   switch (p.comp_dtype) {
     case CKV_F32: e = dispatch_score<CKV_F32>(p, batch, seq_len, max_seq_len, ws, sc, stride, status, stream); break;
     case CKV_BF16: e = dispatch_score<CKV_BF16>(p, batch, seq_len, max_seq_len, ws, sc, stride, status, stream); break;

@@ -1,10 +1,11 @@
 """ckv_decode_step: append, select and attend of one layer in one call.
 
-The fused call runs the same kernels as the three calls except that the append runs beside the
-indexer's query pass (one front kernel on large batches) and that pass also writes the cos/sin
-table of the rotary pairs with the prep kernel's arithmetic, so every result must be bit-identical
-to the three calls': the output, the selection and every byte the append writes. Each side works
-on its own copy of the same generated pools.
+The fused call runs the same kernels as the three calls except that the indexer's query pass runs
+beside the append on sparse layers (and also writes the cos/sin table of the rotary pairs with the
+prep kernel's arithmetic), and that on dense layers of large batches one front kernel runs the
+append beside the attention's query preparation, so every result must be bit-identical to the
+three calls': the output, the selection and every byte the append writes. Each side works on its
+own copy of the same generated pools.
 """
 
 import numpy as np
@@ -19,8 +20,8 @@ pytestmark = pytest.mark.gpu
 
 CACHE_PLANES = ("comp_codes", "comp_scales", "win_codes", "win_scales", "residue_kv", "residue_logit")
 
-# batches of up to 18 requests launch the append and the query pass as two kernels, larger ones as
-# one front kernel (more (request, slice) CTAs than SMs): both forms are covered
+# sparse layers launch the append and the query pass as two kernels; dense layers of more than 18
+# requests (more (request, slice) CTAs than SMs) one front kernel: both forms are covered
 _LENS24 = tuple(1000 + (7919 * i) % 30000 for i in range(24))
 SMALL = [
     S.scaled(S.csa_b8_ctx32k(), (32768, 20001, 4099, 9, 700, 131), "fused", seed=6000),
