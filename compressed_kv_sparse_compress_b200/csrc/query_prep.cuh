@@ -1,8 +1,9 @@
 // Query passes shared by the kernels of the indexer, the attention and the fused decode step's
-// front kernel: the head-averaged query q_bar of the indexer (one slice of dim pairs per call)
-// and the cos/sin table of the rotary pairs at the query position (for the combine's inverse
-// rotation). Each runs on a group of 256 threads (ids tid) that synchronise through barrier
-// bar_id (0 when the group is the whole CTA).
+// front kernel: the head-averaged query q_bar of the indexer's q-bar pass (one slice of dim pairs
+// per call), the cos/sin table of the rotary pairs at the query position (for the combine's
+// inverse rotation; attention prep and the dense front kernel) and a part of the attention's query
+// image (the q-bar pass and the dense front kernel). Each runs on a group of 256 threads (ids tid)
+// that synchronise through barrier bar_id (0 when the group is the whole CTA).
 #pragma once
 
 #include "ckv_internal.h"
