@@ -85,7 +85,11 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   if (k0 >= kl.n_keys) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int i = warp; i < kSimtKeys; i += kSimtThreads / 32) {
+  // key i = thread / 8, resolved by its 8 threads together (the same index and table words) and
+  // loaded by them a pair of dims at a time: every key's dependent loads are in flight at once
+  {
+    static_assert(kSimtThreads == 8 * kSimtKeys, "8 threads per key");
+    const int i = threadIdx.x >> 3, r = threadIdx.x & 7;
     const int64_t kk = k0 + i;
     bool ok = kk < kl.n_keys;
     int64_t row = -1;
@@ -93,7 +97,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     if (ok && kk < kl.n_sel) {
       const int64_t ent = idx ? idx[static_cast<int64_t>(b) * idx_stride + kk] : kk;
       if (ent < 0 || ent >= kl.n_c) {
-        if (lane == 0) atomicOr(status, CKV_DEV_BAD_INDEX);
+        if (r == 0) atomicOr(status, CKV_DEV_BAD_INDEX);
         ok = false;
       } else {
         row = comp_row(p, b, ent, status);
@@ -104,15 +108,17 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     }
     ok = ok && row >= 0;
     if (ok) {
-      for (int pr = lane; pr < D / 2; pr += 32)
+      for (int pr = r; pr < D / 2; pr += 8)
         reinterpret_cast<float2*>(xs + i * D)[pr] = is_win ? win_pair(p, row, pr) : comp_pair(p, row, pr);
     }
-    if (lane == 0) valid[i] = ok;
+    if (r == 0) valid[i] = ok;
   }
   __syncthreads();
 
+  // the query rotated with the cos/sin table of the rotary pairs, which the query pass (or the prep
+  // kernel) wrote before this kernel
   const int first_rope = (D - p.d_r) / 2;
-  const double pos = static_cast<double>(L - 1);
+  const double* rope = ws.rope + static_cast<int64_t>(b) * (p.d_r / 2 + 1) * 2;
   for (int h = warp; h < p.H; h += kSimtThreads / 32) {
     const float* qh = q + (static_cast<int64_t>(b) * p.H + h) * D;
     float2 qv[NPL], ov[NPL];
@@ -121,9 +127,9 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
       const int pr = lane + 32 * k;
       float2 v = reinterpret_cast<const float2*>(qh)[pr];
       if (pr >= first_rope) {
-        double a, c;
-        rope_rotate_pair(v.x, v.y, pos, rope_inv_freq(p, pr - first_rope), false, &a, &c);
-        v = make_float2(static_cast<float>(a), static_cast<float>(c));
+        const double cs = rope[2 * (pr - first_rope)], sn = rope[2 * (pr - first_rope) + 1];
+        const double a0 = v.x, a1 = v.y;
+        v = make_float2(static_cast<float>(a0 * cs - a1 * sn), static_cast<float>(a0 * sn + a1 * cs));
       }
       qv[k] = v;
       ov[k] = make_float2(0.f, 0.f);
