@@ -237,16 +237,24 @@ __global__ void __launch_bounds__(kMhPrepThreads) mh_prep_kernel(LayerParams p, 
 
 // ---------------------------------------------------------------------------- scoring
 
-// Warp roles of the score kernel (256 threads): warp 0 lane 0 loads (TMA for the index rows, bulk
-// copies for the entry scales and the query images), warp 1 lane 0 issues the MMAs, warps 4..7
-// (TMEM lane quarters 0..3, one entry per thread) run the epilogue; warp 2 allocates and frees the
-// tensor memory; otherwise warps 2, 3 and the other lanes only take part in the set-up and the
-// final barrier.
-constexpr int kScoreThreads = 256;
+// Warp roles of the score kernel (128 + 128 G threads, G = 1 or 2 epilogue groups): warp 0 lane 0
+// loads (TMA for the index rows, bulk copies for the entry scales and the query images), warp 1
+// lane 0 issues the MMAs, warps 4..4G+3 (TMEM lane quarters 0..3, one entry per thread) run the
+// epilogue; with G = 2 the first group takes the tiles of accumulator 0 and the second those of
+// accumulator 1, so that two tiles' epilogues overlap. Warp 2 allocates and frees the tensor
+// memory; otherwise warps 2, 3 and the other lanes only take part in the set-up and the final
+// barrier. G = 1 runs 3 CTAs per SM with 3 stages, G = 2 runs 2 CTAs per SM (the register file
+// holds no third) with 4 stages.
+constexpr int kMaxScoreThreads = 384;
+constexpr int kEpiWarps = 8;    // weight slots for the largest G
 constexpr int kTile = 128;      // entries per tile = MMA M
 constexpr int kBoxRows = 64;    // entries per TMA box (one pool block holds 256 / r >= 64 of them)
-constexpr int kStages = 3;      // shared-memory stages of index rows (d_I = 128; 2 for 256)
 constexpr int kMeta = 8;        // slots of per-tile entry scales (> stages + 2 tiles in flight)
+
+__host__ __device__ constexpr int score_threads(int groups) { return 128 + 128 * groups; }
+__host__ __device__ constexpr int score_ctas(int groups) { return groups == 2 ? 2 : 3; }
+// shared-memory stages of index rows: d_I = 128 as above, 2 for d_I = 256
+__host__ __device__ constexpr int score_stages(int dim, int groups) { return dim == 128 ? (groups == 2 ? 4 : 3) : 2; }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -310,22 +318,22 @@ __device__ __forceinline__ void bar_arrive(uint32_t bar) {
 // Shared memory of the score kernel, byte offsets from a 1024-aligned base.
 struct MhSmem {
   uint32_t stage_bytes, stages, a, q, q_bytes, w, meta, mask, bars, tmem, flag, scan, prefix, end_fixed;
-  __host__ __device__ MhSmem(int heads, int dim) {
+  __host__ __device__ MhSmem(int heads, int dim, int groups) {
     stage_bytes = kTile * dim;                         // 128 entries x d_I e4m3
-    stages = dim == 128 ? kStages : 2;
+    stages = score_stages(dim, groups);
     a = 0;
     q = a + stages * stage_bytes;                      // 2 query slots of H_I x d_I e4m3
     q_bytes = static_cast<uint32_t>(heads) * dim;
-    w = q + 2 * ((q_bytes + 1023) / 1024 * 1024);      // float[4 warps][2][128] scaled weights
-    meta = w + 4096;                                   // float[kMeta][128] entry scales
+    w = q + 2 * ((q_bytes + 1023) / 1024 * 1024);      // float[8 warps][2][H] scaled weights
+    meta = w + (kEpiWarps * 2 * 4 * heads + 1023) / 1024 * 1024;  // float[kMeta][128] entry scales
     mask = meta + kMeta * 512;                         // int[kMeta] valid 64-entry runs
     bars = mask + 4 * kMeta;                           // uint64: full[8], empty[8], qfull[2],
                                                        // qempty[2], tfull[2], tempty[2], drain,
                                                        // mfull[kMeta], mempty[kMeta]
     tmem = bars + 8 * (25 + 2 * kMeta);
     flag = tmem + 8;                                   // int abort flag
-    scan = flag + 8;                                   // int32[8]
-    prefix = scan + 32;                                // int32[batch + 1], then n_c [batch]
+    scan = flag + 8;                                   // int32[kMaxScoreThreads / 32]
+    prefix = scan + 4 * (kMaxScoreThreads / 32);       // int32[batch + 1], then n_c [batch]
     end_fixed = prefix;
   }
 };
@@ -362,14 +370,15 @@ struct TileWalk {
   }
 };
 
-template <int DI>
-__global__ void __launch_bounds__(kScoreThreads, 3) mh_score_kernel(const __grid_constant__ CUtensorMap rows_map,
+template <int DI, int G>
+__global__ void __launch_bounds__(score_threads(G), score_ctas(G)) mh_score_kernel(const __grid_constant__ CUtensorMap rows_map,
                                                                      LayerParams p, IndexParams ip, int batch,
                                                                      IndexerWs ws, const uint8_t* qimage,
                                                                      const float* wq, float* scores, int64_t stride,
                                                                      uint32_t tmem_cols, uint32_t* status) {
-  const MhSmem S(ip.heads, DI);
-  constexpr int kNS = DI == 128 ? kStages : 2;
+  constexpr int kScoreThreads = score_threads(G);
+  const MhSmem S(ip.heads, DI, G);
+  constexpr int kNS = score_stages(DI, G);
   constexpr int kChunks = DI / 128;  // 128-byte column chunks of a row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -582,20 +591,22 @@ __global__ void __launch_bounds__(kScoreThreads, 3) mh_score_kernel(const __grid
       if (!mbar_wait(drain, 0)) *abort_flag = 1;
     }
   } else if (warp >= 4) {
-    // ---------------- epilogue: entry j = 32 (warp - 4) + lane = TMEM lane; score, digit count
-    const int q4 = warp - 4;
+    // ---------------- epilogue: entry j = 32 (warp % 4) + lane = TMEM lane; score, digit count.
+    //                  Group eg takes the CTA's tiles it = eg, eg + G, ...
+    const int q4 = warp & 3;
+    const int eg = (warp - 4) >> 2;
     const int j = q4 * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-    float* w_warp = w_sh + q4 * 256;  // this warp's two weight slots
+    float* w_warp = w_sh + (warp - 4) * 2 * H;  // this warp's two weight slots
     int prev_b = -1, ns = 0, qs = 0;
-    int64_t it = 0;
+    int64_t it = eg;
     TileWalk walk(prefix, n_c, batch, t_lo);
-    for (int64_t t = t_lo; t < t_hi && !*abort_flag; ++t, ++it) {
+    for (int64_t t = t_lo + eg; t < t_hi && !*abort_flag; t += G, it += G) {
       const TileInfo ti = walk.at(t);
       if (ti.b != prev_b) {  // this request's scaled head weights into the warp's slot qs
         qs = ns & 1;
         __syncwarp();
-        for (int h = lane; h < H; h += 32) w_warp[qs * 128 + h] = wq[static_cast<int64_t>(ti.b) * H + h];
+        for (int h = lane; h < H; h += 32) w_warp[qs * H + h] = wq[static_cast<int64_t>(ti.b) * H + h];
         __syncwarp();
         prev_b = ti.b;
         ++ns;
@@ -617,7 +628,7 @@ __global__ void __launch_bounds__(kScoreThreads, 3) mh_score_kernel(const __grid
       float sum = 0.f;
       if (ok) {
         const uint32_t taddr = tmem + lane_base + static_cast<uint32_t>(acc) * (tmem_cols / 2);
-        const float4* wv = reinterpret_cast<const float4*>(w_warp + qs * 128);
+        const float4* wv = reinterpret_cast<const float4*>(w_warp + qs * H);
         for (int g = 0; g < H; g += 16) {  // H is a multiple of 16
           uint32_t v[16];
           tmem_ld16(taddr + g, v);
@@ -688,24 +699,28 @@ cudaError_t launch_mh_score(const LayerParams& p, const IndexParams& ip, int bat
           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
       CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const MhSmem S(ip.heads, DI);
-  auto kern = mh_score_kernel<DI>;
+  // Two epilogue groups while the grid gets few tiles per CTA (per 256 K-token request and below:
+  // 32K 14.1 -> 13.2 us, 256K 20.1 -> 18.2 us per launch); one group and 3 CTAs per SM for long
+  // streams (1M: 39.6 against 43.0 us)
+  const int64_t tiles = static_cast<int64_t>(batch) * ((static_cast<int64_t>(max_seq_len) / p.r + kTile - 1) / kTile);
+  const int groups = tiles < static_cast<int64_t>(sm_count()) * 3 * 8 ? 2 : 1;
+  const MhSmem S(ip.heads, DI, groups);
+  auto kern = groups == 2 ? mh_score_kernel<DI, 2> : mh_score_kernel<DI, 1>;
   const uint32_t cols = 2 * ip.heads <= 32 ? 32u : 2 * ip.heads <= 64 ? 64u : 2 * ip.heads <= 128 ? 128u : 256u;
   const int smem = static_cast<int>(S.end_fixed + sizeof(int32_t) * (2 * batch + 1)) + 1024;
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  // CTAs resident per SM: by shared memory (228 KB per SM, 1 KB reserved per CTA) and by tensor
-  // memory (512 columns); a persistent grid of that many per SM
+  // CTAs resident per SM: by shared memory (228 KB per SM, 1 KB reserved per CTA), by tensor
+  // memory (512 columns) and by registers; a persistent grid of that many per SM
   int per_sm = 233472 / (smem + 1024);
   if (per_sm > static_cast<int>(512 / cols)) per_sm = static_cast<int>(512 / cols);
-  if (per_sm > 3) per_sm = 3;
+  if (per_sm > score_ctas(groups)) per_sm = score_ctas(groups);
   if (per_sm < 1) per_sm = 1;
-  const int64_t tiles = static_cast<int64_t>(batch) * ((static_cast<int64_t>(max_seq_len) / p.r + kTile - 1) / kTile);
   int64_t grid = static_cast<int64_t>(sm_count()) * per_sm;
   if (grid > tiles) grid = tiles;
   if (grid < 1) grid = 1;
   prof_begin(kProfScore, stream);
-  e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kScoreThreads), static_cast<size_t>(smem), stream,
+  e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(score_threads(groups)), static_cast<size_t>(smem), stream,
                     map, p, ip, batch, ws, qimage, wq, scores, stride, cols, status);
   prof_end(kProfScore, stream);
   return e;

@@ -92,12 +92,15 @@ def test_mh_scores_and_selection_match_the_oracle(cuda_lib, case):
     _check_against_oracle(w, gen, ix, idx, cnt, sc, k)
 
 
-def test_mh_many_short_requests_per_cta(cuda_lib):
-    # 2048 requests of 1 or 2 tiles (every 7th with no candidate): each persistent CTA walks
-    # several requests, so both query-image slots and the per-warp weight slots are reused and the
-    # producer waits for the MMAs of the request two switches back
-    lens = tuple((512 + 100 * (i % 3)) if i % 7 else 3 for i in range(2048))
-    w = S.Workload("mh_2048req", lens, 64, 512, 64, 128, (S.LayerSpec(4, 16, "bf16", "fp8"),),
+@pytest.mark.parametrize("n,base", [(2048, 512), (1200, 200)], ids=["one_epilogue_group", "two_epilogue_groups"])
+def test_mh_many_short_requests_per_cta(cuda_lib, n, base):
+    # n requests of 1 or 2 tiles (every 7th with no candidate): each persistent CTA walks several
+    # requests, so both query-image slots and the per-warp weight slots are reused and the
+    # producer waits for the MMAs of the request two switches back. 2048 requests of 2 tiles take
+    # the one-group kernel (3 CTAs per SM), 1200 of 1 tile the two-group kernel, whose groups
+    # take alternate tiles and so see alternate requests
+    lens = tuple((base + 100 * (i % 3)) if i % 7 else 3 for i in range(n))
+    w = S.Workload(f"mh_{n}req", lens, 64, 512, 64, 128, (S.LayerSpec(4, 16, "bf16", "fp8"),),
                    paged=True, from_scratch=False, seed=7100)
     gen = S.generate(w, "cuda")
     ix = S.generate_index(w, gen, device="cuda")
